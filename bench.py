@@ -1,0 +1,548 @@
+#!/usr/bin/env python
+"""Throughput of the bit-packed binary-weight x ternary-activation path.
+
+Default workload: the LLaMA-7B-shaped projections (K, N) in {(4096, 4096),
+(4096, 11008), (11008, 4096)} with per-128-column weight scales. One step =
+for each shape: ternarize+pack the decode activations (M=1) and run the GEMV,
+then ternarize+pack the prefill activations (M=2048) and run the tiled GEMM.
+Weights are binarized and packed once, before timing (an offline step).
+
+Metric: effective TOPS = sum over the step's products of 2*M*N*K, divided by
+the device time of the step (CUDA-graph replay, L2 flushed between steps by a
+256 MiB write). With torchrun, every rank runs the same step on its own batch
+(weak scaling, no data-path collective) and the time is the max over ranks.
+
+--impl reference times the CPU oracle (a plain C loop over unpacked values)
+on a bounded row sample of the same workload. --workload selects the other
+measured rows: bert, tiny, attn, billm1, billm16, billm512, pack.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "bit-packed bin x tern GEMM effective TOPS & % roofline at LLaMA-7B shapes"
+UNIT = "TOPS"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ plumbing
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(backend: str):
+    world, rank, local = dist_info()
+    if world > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend, timeout=timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def weak_scaling_value(units_per_rank_step: float, steps: int, world: int, max_seconds: float):
+    """Whole-job throughput: units processed by all ranks / the slowest rank's time."""
+    return units_per_rank_step * steps * world / max_seconds
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows)}
+
+
+class L2Flusher:
+    def __init__(self):
+        self.buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def event_pair():
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+# ------------------------------------------------------------------ workloads
+class LlamaStep:
+    """Decode GEMVs then prefill GEMMs for the three LLaMA-7B projection shapes."""
+
+    def __init__(self, rank: int, M_prefill: int = 2048, M_decode: int = 1):
+        import binarized_transformer_b200 as bt
+        self.bt = bt
+        self.shapes = workloads.LLAMA_SHAPES
+        self.group = workloads.LLAMA_GROUP
+        self.M = {"prefill": M_prefill, "decode": M_decode}
+        self.w = []
+        self.X = {"prefill": [], "decode": []}
+        self.X_host = {"prefill": [], "decode": []}
+        self.planes = {"prefill": [], "decode": []}
+        self.Y = {"prefill": [], "decode": []}
+        for s, (K, N) in enumerate(self.shapes):
+            W = torch.from_numpy(workloads.llama_weights(s)).cuda()
+            self.w.append(bt.bwta_pack_weights(W, self.group))
+            del W
+            for phase in ("decode", "prefill"):
+                M = self.M[phase]
+                Xh = torch.from_numpy(workloads.llama_acts(s, M, stream=rank)).pin_memory()
+                self.X_host[phase].append(Xh)
+                self.X[phase].append(Xh.cuda())
+                ld = bt.ld_words_for(K)
+                self.planes[phase].append((
+                    torch.empty((M, ld), dtype=torch.int32, device="cuda"),
+                    torch.empty((M, ld), dtype=torch.int32, device="cuda"),
+                    torch.empty((M,), dtype=torch.float32, device="cuda")))
+                self.Y[phase].append(torch.empty((M, N), dtype=torch.float32, device="cuda"))
+        self.Y_host = {p: [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in self.Y[p]]
+                       for p in self.Y}
+        torch.cuda.synchronize()
+
+    def launches(self):
+        """(name, callable, ops, alg_bytes) for every kernel launch of one step, in order."""
+        bt = self.bt
+        out = []
+        for phase in ("decode", "prefill"):
+            for s, (K, N) in enumerate(self.shapes):
+                M = self.M[phase]
+                X, (m, sg, sc), Y = self.X[phase][s], self.planes[phase][s], self.Y[phase][s]
+                wb, ws = self.w[s]
+                ld = m.shape[1]
+                G = K // self.group
+                qa_bytes = M * K * 2 + 2 * M * ld * 4 + M * 4
+                out.append((f"quantize_pack_{phase}_{K}x{N}",
+                            lambda X=X, o=(m, sg, sc): bt.bwta_quantize_pack_acts(X, out=o),
+                            0, qa_bytes))
+                gm_bytes = N * ld * 4 + N * G * 4 + 2 * M * ld * 4 + M * 4 + M * N * 4
+                out.append((f"{'gemv' if phase == 'decode' else 'gemm'}_{K}x{N}_M{M}",
+                            lambda m=m, sg=sg, sc=sc, wb=wb, ws=ws, K=K, Y=Y:
+                            bt.bwta_gemm(m, sg, sc, wb, ws, K, self.group, out=(Y, None)),
+                            2 * M * N * K, gm_bytes))
+        return out
+
+    def ops(self):
+        return sum(op for _, _, op, _ in self.launches())
+
+    def run(self):
+        for _, fn, _, _ in self.launches():
+            fn()
+
+    def h2d_bytes(self):
+        return sum(x.numel() * x.element_size() for p in self.X_host for x in self.X_host[p])
+
+    def d2h_bytes(self):
+        return sum(y.numel() * y.element_size() for p in self.Y_host for y in self.Y_host[p])
+
+    def run_e2e(self):
+        """Host fp16 activations in, host fp32 outputs out, through the public API."""
+        for p in ("decode", "prefill"):
+            for s in range(len(self.shapes)):
+                self.X[p][s].copy_(self.X_host[p][s], non_blocking=True)
+        self.run()
+        for p in ("decode", "prefill"):
+            for s in range(len(self.shapes)):
+                self.Y_host[p][s].copy_(self.Y[p][s], non_blocking=True)
+
+
+def capture_graph(fn):
+    """CUDA graph of fn (run once eagerly first so one-time setup stays outside)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
+
+
+def time_steps(step_fn, steps, warmup, flush):
+    """Per-step device time (s) with CUDA events, L2 flushed before each step."""
+    for _ in range(warmup):
+        flush()
+        step_fn()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    total = 0.0
+    per = []
+    for _ in range(steps):
+        flush()
+        a, b = event_pair()
+        a.record()
+        step_fn()
+        b.record()
+        b.synchronize()
+        dt = a.elapsed_time(b) * 1e-3
+        per.append(dt)
+        total += dt
+    torch.cuda.synchronize()
+    barrier()
+    return total, per
+
+
+def per_kernel_times(step, reps, flush):
+    """Average device time of every launch of a step, each bracketed by events
+    on the launching stream (eager launches, L2 flushed before each step)."""
+    launches = step.launches()
+    acc = {name: [] for name, _, _, _ in launches}
+    for _ in range(reps):
+        flush()
+        evs = []
+        for name, fn, _, _ in launches:
+            a, b = event_pair()
+            a.record()
+            fn()
+            b.record()
+            evs.append((name, a, b))
+        torch.cuda.synchronize()
+        for name, a, b in evs:
+            acc[name].append(a.elapsed_time(b) * 1e-3)
+    meta = {name: (op, by) for name, _, op, by in launches}
+    return {name: {"s": statistics.mean(v), "ops": meta[name][0], "bytes": meta[name][1]}
+            for name, v in acc.items()}
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample(rows_per_shape: int = 64):
+    """The CPU oracle on a bounded sample of the LLaMA step: `rows_per_shape`
+    prefill rows per shape plus every decode row. Returns (ops, seconds, cores).
+    Weight binarization is offline on both arms and is not timed."""
+    import oracle
+    oracle.build()
+    prepared = []
+    for s, (K, N) in enumerate(workloads.LLAMA_SHAPES):
+        W = workloads.llama_weights(s)
+        b, alpha = oracle.binarize_weights(W, workloads.LLAMA_GROUP)
+        Xp = workloads.llama_acts(s, 2048)[:rows_per_shape]
+        Xd = workloads.llama_acts(s, 1)
+        prepared.append((b, alpha, Xp, Xd, K, N))
+    ops = 0
+    t0 = time.perf_counter()
+    for b, alpha, Xp, Xd, K, N in prepared:
+        for X in (Xd, Xp):
+            a, sc = oracle.quantize_acts(X)
+            d = oracle.int_dots(a, b, workloads.LLAMA_GROUP)
+            oracle.linear_out(d, alpha, sc)
+            ops += 2 * X.shape[0] * N * K
+    dt = time.perf_counter() - t0
+    return ops, dt, oracle.num_threads()
+
+
+# ------------------------------------------------------------------ main arms
+def run_ours(args):
+    world, rank, local = dist_init("nccl")
+    torch.cuda.set_device(local)
+    import binarized_transformer_b200 as bt
+    from binarized_transformer_b200 import microbench as mb
+    bt.load_library()
+    flush = L2Flusher()
+
+    step = LlamaStep(rank)
+    ops_step = step.ops()
+    n_launch_step = len(step.launches())
+
+    graph = capture_graph(step.run)
+    with ClockSampler(local) as clk:
+        total, per = time_steps(graph.replay, args.steps, args.warmup, flush)
+    tmax = max_over_ranks(total, device="cuda")
+    value = weak_scaling_value(ops_step, args.steps, world, tmax) / 1e12
+
+    # end to end through the public API with host buffers (copies timed)
+    e2e_total, _ = time_steps(step.run_e2e, max(1, args.steps), 1, flush)
+    e2e_max = max_over_ranks(e2e_total, device="cuda")
+    e2e_value = weak_scaling_value(ops_step, max(1, args.steps), world, e2e_max) / 1e12
+
+    kern = per_kernel_times(step, max(3, args.steps), flush)
+
+    if rank != 0:
+        barrier()
+        return
+    peaks, peak_src = measured_peaks()
+    wordop = mb.rate("wordop")          # word-ops / s: LOP3 + POPC + add
+    popc_peak_tops = wordop * 64 / 1e12  # one word-op = 32 MACs = 64 ops
+    gemms = {k: v for k, v in kern.items() if k.startswith("gemm_")}
+    g_ops = sum(v["ops"] for v in gemms.values())
+    g_s = sum(v["s"] for v in gemms.values())
+    achieved = g_ops / g_s / 1e12
+    hbm = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
+    kernels = {}
+    for name, v in kern.items():
+        e = {"us": round(v["s"] * 1e6, 3), "alg_bytes": v["bytes"],
+             "gbs": round(v["bytes"] / v["s"] / 1e9, 1)}
+        if v["ops"]:
+            e["tops"] = round(v["ops"] / v["s"] / 1e12, 2)
+        if name.startswith("gemm_"):
+            e["frac_of_popc_roofline"] = round(v["ops"] / v["s"] / 1e12 / popc_peak_tops, 4)
+        else:
+            e["frac_of_hbm"] = round(v["bytes"] / v["s"] / 1e9 / hbm, 4)
+        kernels[name] = e
+    cpu_ops, cpu_s, cores = oracle_sample(args.cpu_rows)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tmax / args.steps * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u32", "data": "synthetic",
+        "config": {"workload": "llama7b_projections", "shapes_KxN": [list(s) for s in step.shapes],
+                   "M_prefill": step.M["prefill"], "M_decode": step.M["decode"],
+                   "group": step.group, "acts": "student-t(3), 1% x20 outliers, ternarized",
+                   "l2": "flushed before every step (256 MiB write)",
+                   "parallelism": f"dp{world}" if world > 1 else "single"},
+        "roofline": {"bound": "alu", "kernel": "k_gemm_tiled (prefill, 3 shapes)",
+                     "achieved": round(achieved, 3), "peak": round(popc_peak_tops, 3),
+                     "unit": "TOPS", "frac": round(achieved / popc_peak_tops, 4),
+                     "peak_source": "microbenchmarked LOP3+POPC+IADD word-op rate x 64 ops/word",
+                     "traffic": None},
+        "cpu_baseline": {"value": round(cpu_ops / cpu_s / 1e12, 6), "unit": UNIT, "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{args.cpu_rows} prefill rows per shape + the decode row, "
+                                   f"3 LLaMA-7B shapes, {cpu_s:.2f} s"},
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": step.h2d_bytes(),
+                "d2h_bytes_per_step": step.d2h_bytes()},
+        "gpu_launches": n_launch_step * args.steps,
+        "clocks": clk.summary(),
+        "kernels": kernels,
+        "hbm_peak_gbs": hbm, "hbm_peak_source": peak_src,
+        "step_ms": [round(p * 1e3, 4) for p in per],
+    }
+    print(json.dumps(line), flush=True)
+    barrier()
+
+
+def run_reference(args):
+    world, rank, _ = dist_info()
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(max(2, args.cpu_rows // 8))
+    ops = secs = 0.0
+    cores = 1
+    for _ in range(args.steps):
+        o, s, cores = oracle_sample(args.cpu_rows)
+        ops += o
+        secs += s
+    value = ops / secs / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": "llama7b_projections", "group": workloads.LLAMA_GROUP,
+                   "sample_rows_per_shape": args.cpu_rows},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{args.cpu_rows} prefill rows per shape + the decode row per step"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _time_fn(fn, reps, flush):
+    """Mean device time of fn over reps, L2 flushed before each rep."""
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush()
+        a, b = event_pair()
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b) * 1e-3)
+    return statistics.mean(ts)
+
+
+def run_rows(args):
+    """One JSON line per measured row of the other workloads (1 GPU)."""
+    import binarized_transformer_b200 as bt
+    from binarized_transformer_b200 import microbench as mb
+    torch.cuda.set_device(0)
+    flush = L2Flusher()
+    peaks, _ = measured_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
+    popc_tops = mb.rate("wordop") * 64 / 1e12
+    reps = max(3, args.steps)
+    rows = args.workload.split(",")
+    if "all" in rows:
+        rows = ["tiny", "bert", "attn", "billm1", "billm16", "billm512", "pack"]
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    def emit(name, t, ops=None, nbytes=None, **extra):
+        d = {"row": name, "us": round(t * 1e6, 3)}
+        if ops:
+            d["tops"] = round(ops / t / 1e12, 3)
+            d["frac_of_popc_roofline"] = round(ops / t / 1e12 / popc_tops, 4)
+        if nbytes:
+            d["alg_bytes"] = nbytes
+            d["gbs"] = round(nbytes / t / 1e9, 1)
+            d["frac_of_hbm"] = round(nbytes / t / 1e9 / hbm, 4)
+        d.update(extra)
+        print(json.dumps(d), flush=True)
+
+    def linear_rows(tag, X, W, group):
+        M, K = X.shape
+        N = W.shape[0]
+        wb, ws = bt.bwta_pack_weights(dev(W), group)
+        Xd = dev(X)
+        m, sg, sc = bt.bwta_quantize_pack_acts(Xd)
+        Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        ld = m.shape[1]
+        t = _time_fn(lambda: bt.bwta_quantize_pack_acts(Xd, out=(m, sg, sc)), reps, flush)
+        emit(f"{tag}_quantize_pack", t, nbytes=M * K * 2 + 2 * M * ld * 4 + M * 4)
+        G = (K // group) if group else 1
+        t = _time_fn(lambda: bt.bwta_gemm(m, sg, sc, wb, ws, K, group, out=(Y, None)), reps, flush)
+        emit(f"{tag}_gemm", t, ops=2 * M * N * K,
+             nbytes=N * ld * 4 + N * G * 4 + 2 * M * ld * 4 + M * 4 + M * N * 4)
+
+    for row in rows:
+        if row == "tiny":
+            t = workloads.tiny()
+            linear_rows("tiny", t["X"], t["W"], 0)
+        elif row == "bert":
+            for s in (0, 1):
+                t = workloads.bert(s)
+                linear_rows(f"bert{s}_{t['K']}x{t['N']}", t["X"], t["W"], 0)
+        elif row == "attn":
+            a = workloads.attn()
+            B, H, L, D = workloads.ATTN_SHAPE
+            Q, Kt = dev(a["Q"].reshape(-1, D)), dev(a["K"].reshape(-1, D))
+            qm, qs, qsc = bt.bwta_quantize_pack_acts(Q)
+            km, ks, ksc = bt.bwta_quantize_pack_acts(Kt)
+            t = _time_fn(lambda: bt.bwta_quantize_pack_acts(Q, out=(qm, qs, qsc)), reps, flush)
+            emit("attn_quantize_pack_q", t, nbytes=Q.numel() * 2 + 2 * qm.numel() * 4 + qsc.numel() * 4)
+            Si = torch.empty((B * H, L, L), dtype=torch.int32, device="cuda")
+            Sf = torch.empty((B * H, L, L), dtype=torch.float32, device="cuda")
+            inb = 2 * (qm.numel() + km.numel()) * 4 + (qsc.numel() + ksc.numel()) * 4
+            for wi, wf, tag in ((True, True, "both"), (False, True, "f32"), (True, False, "i32")):
+                fn = lambda wi=wi, wf=wf: bt.bwta_attn_scores(
+                    qm, qs, qsc, km, ks, ksc, B * H, L, L, D, want_int=wi, want_float=wf,
+                    out=(Si if wi else None, Sf if wf else None))
+                t = _time_fn(fn, reps, flush)
+                emit(f"attn_scores_{tag}", t, nbytes=inb + Si.numel() * 4 * (int(wi) + int(wf)),
+                     outputs=tag)
+        elif row.startswith("billm"):
+            M = int(row[5:])
+            if not hasattr(run_rows, "_billm"):
+                run_rows._billm = bt.billm_pack_weights(dev(workloads.billm_weights()))
+            Wq = run_rows._billm
+            X = dev(workloads.billm_acts(M))
+            Y = torch.empty((M, Wq.N), dtype=torch.float32, device="cuda")
+            t = _time_fn(lambda: bt.billm_gemm(X, Wq, out=Y), reps, flush)
+            wbytes = sum(x.numel() * x.element_size() for x in (Wq.sign, Wq.gmap, Wq.res, Wq.bscale))
+            emit(f"billm_gemm_M{M}", t, nbytes=wbytes + X.numel() * 2 + Y.numel() * 4,
+                 gflops=round(2 * M * Wq.N * Wq.K / t / 1e9, 1))
+        elif row == "pack":
+            for s, (K, N) in enumerate(workloads.LLAMA_SHAPES):
+                W = dev(workloads.llama_weights(s))
+                t = _time_fn(lambda: bt.bwta_pack_weights(W, 128), reps, flush)
+                emit(f"pack_weights_{K}x{N}", t, nbytes=W.numel() * 4 + W.numel() // 8 + W.numel() // 32)
+            W = dev(workloads.billm_weights())
+            t = _time_fn(lambda: bt.billm_pack_weights(W), 1, flush)
+            emit("billm_pack_weights", t, nbytes=W.numel() * 4)
+        else:
+            raise SystemExit(f"unknown workload row {row}")
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama")
+    ap.add_argument("--cpu-rows", type=int, default=64)
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.workload != "llama":
+        return run_rows(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,247 @@
+"""Python binding of libbwta.so (include/bwta.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libbwta.so. PyTorch provides device memory and the current CUDA
+stream. There is no CPU fallback: importing works anywhere, but every call
+raises if the compiled library is missing or no CUDA device is present.
+
+Bit planes are returned as int32 tensors holding the uint32 words
+(bit i of word w is element 32*w + i).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbwta.so")
+MB_LIB_PATH = os.path.join(_HERE, "libbwta_microbench.so")
+
+BWTA_OK, BWTA_ERR_INVALID_ARG, BWTA_ERR_UNSUPPORTED, BWTA_ERR_ALIGNMENT, BWTA_ERR_CUDA = range(5)
+STATUS_NONFINITE, STATUS_TIMEOUT = 0x1, 0x2
+TERNARY, BINARY = 0, 1
+ERROR_NAMES = {1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA"}
+
+EXPORTS = ["bwta_pack_weights", "bwta_quantize_pack_acts", "bwta_gemm", "bwta_attn_scores",
+           "billm_pack_weights", "billm_gemm", "bwta_version"]
+
+
+class BwtaError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} returned {code} ({ERROR_NAMES.get(code, '?')})")
+        self.code = code
+
+
+class BillmWeightsC(C.Structure):
+    _fields_ = [("sign", C.c_void_p), ("gmap", C.c_void_p), ("res", C.c_void_p),
+                ("sal", C.c_void_p), ("bscale", C.c_void_p), ("N", C.c_int64),
+                ("K", C.c_int64), ("ldw_words", C.c_int64), ("block", C.c_int64),
+                ("n_sal", C.c_int64)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libbwta.so (raises FileNotFoundError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FileNotFoundError(f"{path} is missing: run `python -m binarized_transformer_b200.build`")
+    lib = C.CDLL(path)
+    vp, i64, ci, cf = C.c_void_p, C.c_int64, C.c_int, C.c_float
+    lib.bwta_pack_weights.argtypes = [vp, i64, i64, i64, i64, vp, i64, vp, vp, vp]
+    lib.bwta_quantize_pack_acts.argtypes = [vp, i64, i64, i64, ci, cf, vp, vp, i64, vp, vp, vp]
+    lib.bwta_gemm.argtypes = [vp, vp, vp, i64, i64, vp, vp, i64, i64, i64, i64, vp, i64, vp, i64,
+                              vp, vp]
+    lib.bwta_attn_scores.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp, vp]
+    lib.billm_pack_weights.argtypes = [vp, i64, ci, C.POINTER(BillmWeightsC), vp, vp]
+    lib.billm_gemm.argtypes = [vp, i64, i64, C.POINTER(BillmWeightsC), vp, i64, vp, vp]
+    lib.bwta_version.restype = C.c_char_p
+    for name in EXPORTS[:-1]:
+        getattr(lib, name).restype = C.c_int
+    _lib = lib
+    return lib
+
+
+def _L():
+    if not torch.cuda.is_available():
+        raise RuntimeError("libbwta needs a CUDA device; there is no CPU fallback")
+    return load_library()
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != BWTA_OK:
+        raise BwtaError(fn, rc)
+
+
+def _row_stride(t: torch.Tensor) -> int:
+    """Leading dimension of a row-major 2-D tensor (a single row may carry any stride)."""
+    return t.stride(0) if t.shape[0] > 1 else t.shape[1]
+
+
+def ld_words_for(K: int) -> int:
+    """Smallest legal row stride in words: ceil(K/32) rounded up to a multiple of 4."""
+    return ((K + 31) // 32 + 3) // 4 * 4
+
+
+def new_status(device=None):
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def version() -> str:
+    return load_library().bwta_version().decode()
+
+
+# ------------------------------------------------------------------ BWTA
+def bwta_pack_weights(W: torch.Tensor, group: int = 0, ld_words: int | None = None,
+                      status: torch.Tensor | None = None):
+    """fp32 W [N, K] (cuda) -> (wbits int32 [N, ld_words], wscale fp32 [N, G])."""
+    lib = _L()
+    assert W.is_cuda and W.dtype == torch.float32 and W.dim() == 2 and W.stride(1) == 1
+    N, K = W.shape
+    ld = ld_words or ld_words_for(K)
+    G = -(-K // group) if group else 1
+    wbits = torch.empty((N, ld), dtype=torch.int32, device=W.device)
+    wscale = torch.empty((N, G), dtype=torch.float32, device=W.device)
+    _check("bwta_pack_weights", lib.bwta_pack_weights(
+        _ptr(W), N, K, _row_stride(W), group, _ptr(wbits), ld, _ptr(wscale), _ptr(status), _stream()))
+    return wbits, wscale
+
+
+def bwta_quantize_pack_acts(X: torch.Tensor, mode: int = TERNARY, thresh_ratio: float = 0.5,
+                            ld_words: int | None = None, status: torch.Tensor | None = None,
+                            out=None):
+    """fp16 X [M, K] (cuda) -> (mask int32 [M, ld], sign int32 [M, ld], scale fp32 [M])."""
+    lib = _L()
+    assert X.is_cuda and X.dtype == torch.float16 and X.dim() == 2 and X.stride(1) == 1
+    M, K = X.shape
+    ld = ld_words or ld_words_for(K)
+    if out is None:
+        mask = torch.empty((M, ld), dtype=torch.int32, device=X.device)
+        sign = torch.empty((M, ld), dtype=torch.int32, device=X.device)
+        scale = torch.empty((M,), dtype=torch.float32, device=X.device)
+    else:
+        mask, sign, scale = out
+    _check("bwta_quantize_pack_acts", lib.bwta_quantize_pack_acts(
+        _ptr(X), M, K, _row_stride(X), mode, thresh_ratio, _ptr(mask), _ptr(sign), ld, _ptr(scale),
+        _ptr(status), _stream()))
+    return mask, sign, scale
+
+
+def bwta_gemm(a_mask, a_sign, a_scale, wbits, wscale, K: int, group: int = 0,
+              want_y: bool = True, want_dots: bool = False, status=None, out=None):
+    """Bit-packed GEMM. Returns (Y fp32 [M, N] or None, dots int32 [M, N] or None)."""
+    lib = _L()
+    M, lda = a_mask.shape
+    N, ldw = wbits.shape
+    if out is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=a_mask.device) if want_y else None
+        D = torch.empty((M, N), dtype=torch.int32, device=a_mask.device) if want_dots else None
+    else:
+        Y, D = out
+    _check("bwta_gemm", lib.bwta_gemm(
+        _ptr(a_mask), _ptr(a_sign), _ptr(a_scale), M, lda, _ptr(wbits), _ptr(wscale), N, ldw, K,
+        group, _ptr(Y), _row_stride(Y) if Y is not None else N, _ptr(D),
+        _row_stride(D) if D is not None else N, _ptr(status), _stream()))
+    return Y, D
+
+
+def bwta_attn_scores(q_mask, q_sign, q_scale, k_mask, k_sign, k_scale, BH: int, Lq: int, Lk: int,
+                     D: int, want_int: bool = True, want_float: bool = True, out=None):
+    """Ternary Q.K^T scores. Returns (S int32 [BH, Lq, Lk] or None, S fp32 or None)."""
+    lib = _L()
+    ld = q_mask.shape[-1]
+    dev = q_mask.device
+    if out is None:
+        Si = torch.empty((BH, Lq, Lk), dtype=torch.int32, device=dev) if want_int else None
+        Sf = torch.empty((BH, Lq, Lk), dtype=torch.float32, device=dev) if want_float else None
+    else:
+        Si, Sf = out
+    _check("bwta_attn_scores", lib.bwta_attn_scores(
+        _ptr(q_mask), _ptr(q_sign), _ptr(q_scale), _ptr(k_mask), _ptr(k_sign), _ptr(k_scale),
+        BH, Lq, Lk, D, ld, _ptr(Si), _ptr(Sf), _stream()))
+    return Si, Sf
+
+
+# ------------------------------------------------------------------ BiLLM
+@dataclass
+class BillmWeights:
+    sign: torch.Tensor     # int32 [N, ldw]
+    gmap: torch.Tensor     # int32 [N, ldw]
+    res: torch.Tensor      # uint8 [N, K/block]
+    sal: torch.Tensor      # uint8 [K/block, n_sal]
+    bscale: torch.Tensor   # fp32 [N, K/block, 4]
+    N: int
+    K: int
+    block: int = 128
+    n_sal: int = 8
+
+    @property
+    def ldw(self) -> int:
+        return self.sign.shape[1]
+
+    def cstruct(self) -> BillmWeightsC:
+        return BillmWeightsC(self.sign.data_ptr(), self.gmap.data_ptr(), self.res.data_ptr(),
+                             self.sal.data_ptr() if self.sal.numel() else None,
+                             self.bscale.data_ptr(), self.N, self.K, self.ldw, self.block,
+                             self.n_sal)
+
+    @staticmethod
+    def empty(N: int, K: int, n_sal: int = 8, block: int = 128, device="cuda"):
+        ld = ld_words_for(K)
+        nb = K // block
+        return BillmWeights(
+            sign=torch.empty((N, ld), dtype=torch.int32, device=device),
+            gmap=torch.empty((N, ld), dtype=torch.int32, device=device),
+            res=torch.empty((N, nb), dtype=torch.uint8, device=device),
+            sal=torch.empty((nb, n_sal), dtype=torch.uint8, device=device),
+            bscale=torch.empty((N, nb, 4), dtype=torch.float32, device=device),
+            N=N, K=K, block=block, n_sal=n_sal)
+
+
+def billm_pack_weights(W: torch.Tensor, n_sal: int = 8, split: bool = True, block: int = 128,
+                       status=None) -> BillmWeights:
+    """Latent fp32 W [N, K] (cuda) -> packed BiLLM weights, built on the GPU."""
+    lib = _L()
+    assert W.is_cuda and W.dtype == torch.float32 and W.dim() == 2 and W.stride(1) == 1
+    N, K = W.shape
+    out = BillmWeights.empty(N, K, n_sal, block, W.device)
+    cs = out.cstruct()
+    _check("billm_pack_weights", lib.billm_pack_weights(
+        _ptr(W), _row_stride(W), int(bool(split)), C.byref(cs), _ptr(status), _stream()))
+    return out
+
+
+def billm_gemm(X: torch.Tensor, Wq: BillmWeights, status=None, out=None) -> torch.Tensor:
+    """fp16 X [M, K] x BiLLM weights -> Y fp32 [M, N]."""
+    lib = _L()
+    assert X.is_cuda and X.dtype == torch.float16 and X.dim() == 2 and X.stride(1) == 1
+    M = X.shape[0]
+    Y = out if out is not None else torch.empty((M, Wq.N), dtype=torch.float32, device=X.device)
+    cs = Wq.cstruct()
+    _check("billm_gemm", lib.billm_gemm(_ptr(X), M, _row_stride(X), C.byref(cs), _ptr(Y),
+                                        _row_stride(Y), _ptr(status), _stream()))
+    return Y
+
+
+# ------------------------------------------------------------------ helpers
+def as_u32(t: torch.Tensor):
+    """A bit-plane tensor (int32 on any device) as a numpy uint32 array."""
+    return t.detach().cpu().numpy().view("uint32")
+
+
+def half_from_numpy(x, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(x).to(device)

@@ -1,0 +1,134 @@
+// abi.cu -- the extern "C" entry points of libbwta.so (declared in
+// include/bwta.h): argument validation on the host, then one or two kernel
+// launches on the caller's stream. Nothing here allocates memory.
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+
+using namespace bwta;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? BWTA_OK : BWTA_ERR_CUDA; }
+
+int64_t words_for(int64_t K) { return (K + 31) / 32; }
+
+int check_plane(const void *p, int64_t rows, int64_t ld, int64_t K) {
+  if (rows > 0 && !p) return BWTA_ERR_INVALID_ARG;
+  if (ld < words_for(K)) return BWTA_ERR_INVALID_ARG;
+  if (ld % 4 != 0 || !aligned16(p)) return BWTA_ERR_ALIGNMENT;
+  return BWTA_OK;
+}
+
+int check_group(int64_t group) {
+  if (group < 0) return BWTA_ERR_INVALID_ARG;
+  if (group != 0 && group % 128 != 0) return BWTA_ERR_UNSUPPORTED;
+  return BWTA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *bwta_version(void) { return "bwta 0.1 sm_100a"; }
+
+int bwta_pack_weights(const float *W, int64_t N, int64_t K, int64_t ldW, int64_t group,
+                      uint32_t *wbits, int64_t ldw_words, float *wscale, int32_t *d_status,
+                      bwta_stream_t stream) {
+  if (N < 0 || K <= 0 || ldW < K) return BWTA_ERR_INVALID_ARG;
+  if (int r = check_group(group)) return r;
+  if (N > 0 && (!W || !wscale)) return BWTA_ERR_INVALID_ARG;
+  if (int r = check_plane(wbits, N, ldw_words, K)) return r;
+  return cuda_status(launch_pack_weights(W, N, K, ldW, group, wbits, ldw_words, wscale, d_status,
+                                         (cudaStream_t)stream));
+}
+
+int bwta_quantize_pack_acts(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
+                            float thresh_ratio, uint32_t *mask, uint32_t *sign,
+                            int64_t lda_words, float *scale, int32_t *d_status,
+                            bwta_stream_t stream) {
+  if (M < 0 || K <= 0 || ldX < K) return BWTA_ERR_INVALID_ARG;
+  if (mode != BWTA_TERNARY && mode != BWTA_BINARY) return BWTA_ERR_INVALID_ARG;
+  if (thresh_ratio != 0.5f || K > BWTA_MAX_K) return BWTA_ERR_UNSUPPORTED;
+  if (M > 0 && (!X || !scale)) return BWTA_ERR_INVALID_ARG;
+  if (int r = check_plane(mask, M, lda_words, K)) return r;
+  if (int r = check_plane(sign, M, lda_words, K)) return r;
+  return cuda_status(launch_quantize_pack_acts(X, M, K, ldX, mode, mask, sign, lda_words, scale,
+                                               d_status, (cudaStream_t)stream));
+}
+
+int bwta_gemm(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_scale, int64_t M,
+              int64_t lda_words, const uint32_t *wbits, const float *wscale, int64_t N,
+              int64_t ldw_words, int64_t K, int64_t group, float *Y, int64_t ldY, int32_t *dots,
+              int64_t ldD, int32_t *d_status, bwta_stream_t stream) {
+  if (M < 0 || N < 0 || K <= 0) return BWTA_ERR_INVALID_ARG;
+  if (K > BWTA_MAX_K) return BWTA_ERR_UNSUPPORTED;
+  if (int r = check_group(group)) return r;
+  if (!Y && !dots) return BWTA_ERR_INVALID_ARG;
+  if (Y && ldY < N) return BWTA_ERR_INVALID_ARG;
+  if (dots && ldD < N) return BWTA_ERR_INVALID_ARG;
+  if (M > 0 && !a_scale) return BWTA_ERR_INVALID_ARG;
+  if (N > 0 && !wscale) return BWTA_ERR_INVALID_ARG;
+  if (int r = check_plane(a_mask, M, lda_words, K)) return r;
+  if (int r = check_plane(a_sign, M, lda_words, K)) return r;
+  if (int r = check_plane(wbits, N, ldw_words, K)) return r;
+  if (M == 0 || N == 0) return BWTA_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (gemv_fits(M, lda_words, K, group))
+    return cuda_status(launch_gemv(a_mask, a_sign, a_scale, M, lda_words, wbits, wscale, N,
+                                   ldw_words, K, group, Y, ldY, dots, ldD, s));
+  return cuda_status(launch_gemm_tiled(a_mask, a_sign, a_scale, M, lda_words, wbits, wscale, N,
+                                       ldw_words, K, group, Y, ldY, dots, ldD, d_status, s));
+}
+
+int bwta_attn_scores(const uint32_t *q_mask, const uint32_t *q_sign, const float *q_scale,
+                     const uint32_t *k_mask, const uint32_t *k_sign, const float *k_scale,
+                     int64_t BH, int64_t Lq, int64_t Lk, int64_t D, int64_t ld_words,
+                     int32_t *S_i32, float *S_f32, bwta_stream_t stream) {
+  if (BH < 0 || Lq < 0 || Lk < 0 || D <= 0) return BWTA_ERR_INVALID_ARG;
+  if (!S_i32 && !S_f32) return BWTA_ERR_INVALID_ARG;
+  if (ld_words > 32) return BWTA_ERR_UNSUPPORTED;
+  if (int r = check_plane(q_mask, BH * Lq, ld_words, D)) return r;
+  if (int r = check_plane(q_sign, BH * Lq, ld_words, D)) return r;
+  if (int r = check_plane(k_mask, BH * Lk, ld_words, D)) return r;
+  if (int r = check_plane(k_sign, BH * Lk, ld_words, D)) return r;
+  if (S_f32 && BH * Lq > 0 && !q_scale) return BWTA_ERR_INVALID_ARG;
+  if (S_f32 && BH * Lk > 0 && !k_scale) return BWTA_ERR_INVALID_ARG;
+  if ((S_i32 && !aligned16(S_i32)) || (S_f32 && !aligned16(S_f32))) return BWTA_ERR_ALIGNMENT;
+  return cuda_status(launch_attn_scores(q_mask, q_sign, q_scale, k_mask, k_sign, k_scale, BH, Lq,
+                                        Lk, ld_words, S_i32, S_f32, (cudaStream_t)stream));
+}
+
+static int check_billm(const billm_weights *W) {
+  if (!W) return BWTA_ERR_INVALID_ARG;
+  if (W->N < 0 || W->K <= 0) return BWTA_ERR_INVALID_ARG;
+  if (W->block != 128 || W->K % 128 != 0 || W->n_sal < 0 || W->n_sal > 8)
+    return BWTA_ERR_UNSUPPORTED;
+  if (W->N > 0 && (!W->res || !W->bscale)) return BWTA_ERR_INVALID_ARG;
+  if (W->n_sal > 0 && !W->sal) return BWTA_ERR_INVALID_ARG;
+  if (int r = check_plane(W->sign, W->N, W->ldw_words, W->K)) return r;
+  if (int r = check_plane(W->gmap, W->N, W->ldw_words, W->K)) return r;
+  if (!aligned16(W->bscale)) return BWTA_ERR_ALIGNMENT;
+  return BWTA_OK;
+}
+
+int billm_pack_weights(const float *W, int64_t ldW, int split, const billm_weights *out,
+                       int32_t *d_status, bwta_stream_t stream) {
+  if (int r = check_billm(out)) return r;
+  if (ldW < out->K || (out->N > 0 && !W)) return BWTA_ERR_INVALID_ARG;
+  if (out->N > 0 && (out->n_sal == 0 ? false : !out->sal)) return BWTA_ERR_INVALID_ARG;
+  return cuda_status(launch_billm_pack(W, ldW, split, out, d_status, (cudaStream_t)stream));
+}
+
+int billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W, float *Y,
+               int64_t ldY, int32_t *d_status, bwta_stream_t stream) {
+  if (int r = check_billm(W)) return r;
+  if (M < 0 || ldX < W->K || ldY < W->N) return BWTA_ERR_INVALID_ARG;
+  if (M > 0 && (!X || !Y)) return BWTA_ERR_INVALID_ARG;
+  if (W->K > 40960) return BWTA_ERR_UNSUPPORTED;
+  return cuda_status(launch_billm_gemm(X, M, ldX, W, Y, ldY, d_status, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,186 @@
+/*
+ * bwta.h -- C ABI of libbwta.so: bit-packed binary weights x binary/ternary
+ * activations (BWTA) and BiLLM-format binary weights x fp16 activations, as
+ * hand-written CUDA kernels for NVIDIA B200 (sm_100a).
+ *
+ * Sources:
+ *  "BWTA: Accurate and Efficient Binarized Transformer by Algorithm-Hardware
+ *   Co-design" (abstract, "Core claim", Figure 6): binary weights, ternary
+ *   activations made by projecting tiny values to zero, 32 fp16 values packed
+ *   into one 32-bit word, binary/ternary MatMul for linear and attention.
+ *  "BiLLM: Pushing the Limit of Post-Training Quantization for LLMs"
+ *   (abstract, "Approach", "Limitations"): salient columns with residual
+ *   binarization, non-salient weights split into two groups with their own
+ *   scales, a 1-bit group map; 128-column blocks.
+ *
+ * Conventions shared by every call
+ *  - Bit planes are uint32 words; bit i of word w is element k = 32*w + i.
+ *    Rows of a plane are ld_words apart; ld_words >= ceil(K/32) and
+ *    ld_words % 4 == 0 (16-byte rows). Packers write every word of the row,
+ *    the padding words past K as zero.
+ *  - Sign bit 1 means negative. Mask bit 1 means the ternary value is nonzero;
+ *    sign bits are 0 wherever the mask bit is 0. sign(0) = +1 and -0.0 is 0.
+ *  - Ternary activations: keep x iff |x| > 0.5 * mean|x| over the row (equal
+ *    values are projected to zero); the row scale is the mean |x| over the kept
+ *    entries (0 if none). The test is done exactly in integers (every fp16 is a
+ *    multiple of 2^-24), so the planes do not depend on summation order.
+ *  - Binary weights: b = sign(w); scale = mean|w| per row (group == 0) or per
+ *    `group` consecutive columns (group a positive multiple of 128; the last
+ *    group may be shorter when K is not a multiple of group).
+ *  - Scales are fp32; fp16 data is passed as raw uint16 bit patterns.
+ *  - Ownership: the caller allocates every buffer (device memory unless stated
+ *    otherwise) and keeps it alive until the stream reaches the call. The
+ *    library allocates no memory and keeps no state between calls.
+ *  - Every call is asynchronous on `stream` (NULL = the legacy default stream)
+ *    and returns a bwta_status. Argument checks happen on the host before any
+ *    launch. Data-dependent conditions (non-finite inputs) are reported by
+ *    OR-ing BWTA_STATUS_* flags into *d_status (a device int32, may be NULL);
+ *    kernels never trap.
+ *  - Pointers to bit planes, scales and outputs must be 16-byte aligned;
+ *    fp16/fp32 input matrices must be 16-byte aligned with ld % 8 == 0 (fp16)
+ *    or ld % 4 == 0 (fp32).
+ */
+#ifndef BWTA_H
+#define BWTA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *bwta_stream_t; /* the same type as cudaStream_t */
+
+typedef enum bwta_status {
+  BWTA_OK = 0,
+  BWTA_ERR_INVALID_ARG = 1, /* NULL where a buffer is required, negative size, ld too small */
+  BWTA_ERR_UNSUPPORTED = 2, /* an option or size outside what this version implements */
+  BWTA_ERR_ALIGNMENT = 3,   /* a pointer or leading dimension breaks the alignment rules */
+  BWTA_ERR_CUDA = 4         /* the CUDA runtime reported an error at launch */
+} bwta_status;
+
+/* device-side status flags, OR-ed into *d_status */
+#define BWTA_STATUS_NONFINITE 0x1 /* an input held Inf or NaN; outputs of that row are unspecified */
+#define BWTA_STATUS_TIMEOUT 0x2   /* a bounded wait inside a kernel gave up; outputs are unspecified */
+
+#define BWTA_TERNARY 0
+#define BWTA_BINARY 1
+
+#define BWTA_MAX_K (1 << 22) /* exactness bound of the integer threshold test */
+
+/* Binarize and pack weights (BWTA abstract: binary weights; scale mean|w|).
+ *  W       fp32 [N][ldW] latent weights (read only)
+ *  group   0 (one scale per row) or a positive multiple of 128
+ *  wbits   uint32 [N][ldw_words] out: sign planes
+ *  wscale  fp32 [N][G] out, G = group ? ceil(K/group) : 1; each scale is the
+ *          fp64 sum of |w| in ascending column order divided by the count,
+ *          rounded once to fp32
+ *  Errors: INVALID_ARG, UNSUPPORTED (group), ALIGNMENT; NONFINITE flag. */
+int bwta_pack_weights(const float *W, int64_t N, int64_t K, int64_t ldW, int64_t group,
+                      uint32_t *wbits, int64_t ldw_words, float *wscale, int32_t *d_status,
+                      bwta_stream_t stream);
+
+/* Ternarize (or binarize) and pack activations, one fused pass per row
+ * (BWTA abstract: tiny values projected to zero; Figure 6: 32 fp16 -> one word).
+ *  X            fp16 bits [M][ldX]
+ *  mode         BWTA_TERNARY or BWTA_BINARY (binary: mask all ones for k < K,
+ *               scale = mean|x| over the row)
+ *  thresh_ratio must be 0.5 (the threshold is thresh_ratio * mean|x|)
+ *  mask, sign   uint32 [M][lda_words] out
+ *  scale        fp32 [M] out
+ *  Errors: INVALID_ARG, UNSUPPORTED (ratio, K > BWTA_MAX_K), ALIGNMENT;
+ *  NONFINITE flag. */
+int bwta_quantize_pack_acts(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
+                            float thresh_ratio, uint32_t *mask, uint32_t *sign,
+                            int64_t lda_words, float *scale, int32_t *d_status,
+                            bwta_stream_t stream);
+
+/* Bit-packed GEMM: Y = (s_a * A_ternary) x (alpha * B_binary)^T
+ * (BWTA abstract: the bit-packed binary/ternary MatMul for linear layers).
+ * Per output (m, n) and weight group g over the words of that group:
+ *     d_g = sum popc(mask) - 2 * popc(mask & (a_sign ^ w_sign))
+ *     Y[m][n] = fp32: acc = 0; for g ascending: acc = fma((float)d_g, alpha[n][g], acc);
+ *               Y = acc * a_scale[m]
+ *     dots[m][n] = sum_g d_g  (exact int32)
+ * M <= 8 runs the decode GEMV kernel (its fp32 sum over groups is a tree, not
+ * the serial order above; its dots are the same integers), larger M the tiled
+ * GEMM, which follows the serial order exactly.
+ *  a_mask, a_sign  uint32 [M][lda_words]; a_scale fp32 [M]
+ *  wbits           uint32 [N][ldw_words]; wscale fp32 [N][G]
+ *  Y               fp32 [M][ldY] out, may be NULL
+ *  dots            int32 [M][ldD] out, may be NULL (not both NULL); with group > 0
+ *                  the full-K dots come from a second, ungrouped pass
+ *  d_status        device int32, may be NULL: BWTA_STATUS_TIMEOUT if a bounded
+ *                  wait on a shared-memory barrier gave up
+ *  Errors: INVALID_ARG, UNSUPPORTED (group, K), ALIGNMENT, CUDA. */
+int bwta_gemm(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_scale, int64_t M,
+              int64_t lda_words, const uint32_t *wbits, const float *wscale, int64_t N,
+              int64_t ldw_words, int64_t K, int64_t group, float *Y, int64_t ldY, int32_t *dots,
+              int64_t ldD, int32_t *d_status, bwta_stream_t stream);
+
+/* Ternary attention scores Q . K^T per batch*head (BWTA abstract: binary /
+ * ternary MatMul for the attention operators). Both operands come from
+ * bwta_quantize_pack_acts over rows of length D.
+ *  q_mask, q_sign [BH*Lq][ld_words], q_scale [BH*Lq]
+ *  k_mask, k_sign [BH*Lk][ld_words], k_scale [BH*Lk]
+ *  S_i32 int32 [BH][Lq][Lk] out (may be NULL): S = popc(mq & mk) - 2*popc(mq & mk & (sq ^ sk))
+ *  S_f32 fp32  [BH][Lq][Lk] out (may be NULL): ((float)S * q_scale) * k_scale
+ *  No 1/sqrt(D) and no softmax. Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+int bwta_attn_scores(const uint32_t *q_mask, const uint32_t *q_sign, const float *q_scale,
+                     const uint32_t *k_mask, const uint32_t *k_sign, const float *k_scale,
+                     int64_t BH, int64_t Lq, int64_t Lk, int64_t D, int64_t ld_words,
+                     int32_t *S_i32, float *S_f32, bwta_stream_t stream);
+
+/* BiLLM packed weights (BiLLM "Approach" and "Limitations"). Per block j of
+ * `block` = 128 columns and row n:
+ *  sign   uint32 [N][ldw_words]  1 = negative (b for non-salient, b1 for salient)
+ *  gmap   uint32 [N][ldw_words]  1 = sparse group (0 at salient columns)
+ *  res    uint8  [N][K/block]    bit i: 1 = b2 of salient column sal[j][i] negative
+ *  sal    uint8  [K/block][n_sal] salient columns of block j, ascending
+ *  bscale fp32   [N][K/block][4] (alpha_c, alpha_sp, alpha1, alpha2)
+ * Dequantized weight: alpha_c*b (concentrated), alpha_sp*b (sparse),
+ * alpha1*b1 + alpha2*b2 (salient). */
+typedef struct billm_weights {
+  const uint32_t *sign;
+  const uint32_t *gmap;
+  const uint8_t *res;
+  const uint8_t *sal;
+  const float *bscale;
+  int64_t N, K, ldw_words, block, n_sal;
+} billm_weights;
+
+/* Build the BiLLM packed weights from latent fp32 weights on the GPU.
+ *  Salient columns: per block, the n_sal columns with the largest sum_n w^2
+ *  (fp64, rows ascending; the Hessian of the pages' metric taken as the
+ *  identity, as no calibration data is used); ties go to the lower column.
+ *  Salient weights: alpha1 = mean|w|, b1 = sign(w), r = w - alpha1*b1,
+ *  alpha2 = mean|r|, b2 = sign(r). Other weights: break-point
+ *  p = 0.5*max|w| over the row's non-salient weights in the block; the sparse
+ *  group is |w| > p (only if split != 0); alpha = mean|w| per group (0 if
+ *  empty). Every mean is an fp64 sum in ascending column order divided by the
+ *  count and rounded once to fp32.
+ *  W fp32 [N][ldW]; out: the buffers of `out` (cast away const; device memory).
+ *  block must be 128; 0 <= n_sal <= 8; K % 128 == 0.
+ *  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; NONFINITE flag. */
+int billm_pack_weights(const float *W, int64_t ldW, int split, const billm_weights *out,
+                       int32_t *d_status, bwta_stream_t stream);
+
+/* BiLLM-format GEMM: Y[m][n] = sum_k x[m][k] * what[n][k] with fp32
+ * accumulation, evaluated per block as
+ *   alpha_c*sum_C b x + alpha_sp*sum_S b x + alpha1*sum_sal b1 x + alpha2*sum_sal b2 x.
+ *  X   fp16 bits [M][ldX]
+ *  W   host pointer to a billm_weights whose buffers are device memory
+ *  Y   fp32 [M][ldY] out
+ *  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; NONFINITE flag. */
+int billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W, float *Y,
+               int64_t ldY, int32_t *d_status, bwta_stream_t stream);
+
+/* Library version string, e.g. "bwta 0.1 sm_100a". */
+const char *bwta_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BWTA_H */
