@@ -14,7 +14,8 @@ the device time of the step (CUDA-graph replay, L2 flushed between steps by a
 
 --impl reference times the CPU oracle (a plain C loop over unpacked values)
 on a bounded row sample of the same workload. --workload selects the other
-measured rows: bert, tiny, attn, billm1, billm16, billm512, pack.
+measured rows: llama_prefill, llama_decode, bert, tiny, attn, billm1, billm16,
+billm512, pack (comma separated, or all).
 """
 from __future__ import annotations
 
@@ -480,7 +481,12 @@ def run_rows(args):
              nbytes=N * ld * 4 + N * G * 4 + 2 * M * ld * 4 + M * 4 + M * N * 4)
 
     for row in rows:
-        if row == "tiny":
+        if row in ("llama_prefill", "llama_decode"):
+            M = 2048 if row == "llama_prefill" else 1
+            for s in range(3):
+                t = workloads.llama(s, M)
+                linear_rows(f"llama{s}_{t['K']}x{t['N']}_M{M}", t["X"], t["W"], t["group"])
+        elif row == "tiny":
             t = workloads.tiny()
             linear_rows("tiny", t["X"], t["W"], 0)
         elif row == "bert":
