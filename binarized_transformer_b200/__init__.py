@@ -25,8 +25,10 @@ STATUS_NONFINITE, STATUS_TIMEOUT = 0x1, 0x2
 TERNARY, BINARY = 0, 1
 ERROR_NAMES = {1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA"}
 
-EXPORTS = ["bwta_pack_weights", "bwta_quantize_pack_acts", "bwta_gemm", "bwta_attn_scores",
-           "billm_pack_weights", "billm_gemm", "bwta_version"]
+EXPORTS = ["bwta_pack_weights", "bwta_quantize_pack_acts", "bwta_gemm", "bwta_gemm_ex",
+           "bwta_linear_decode", "bwta_attn_scores", "billm_pack_weights", "billm_gemm",
+           "bwta_version"]
+GEMM_WEIGHTS_READY = 0x1
 
 
 class BwtaError(RuntimeError):
@@ -58,6 +60,10 @@ def load_library(path: str = LIB_PATH):
     lib.bwta_quantize_pack_acts.argtypes = [vp, i64, i64, i64, ci, cf, vp, vp, i64, vp, vp, vp]
     lib.bwta_gemm.argtypes = [vp, vp, vp, i64, i64, vp, vp, i64, i64, i64, i64, vp, i64, vp, i64,
                               vp, vp]
+    lib.bwta_gemm_ex.argtypes = [vp, vp, vp, i64, i64, vp, vp, i64, i64, i64, i64, vp, i64, vp,
+                                 i64, C.c_uint32, vp, vp]
+    lib.bwta_linear_decode.argtypes = [vp, i64, i64, i64, ci, cf, vp, vp, i64, i64, i64, vp, i64,
+                                       vp, i64, C.c_uint32, vp, vp]
     lib.bwta_attn_scores.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp, vp]
     lib.billm_pack_weights.argtypes = [vp, i64, ci, C.POINTER(BillmWeightsC), vp, vp]
     lib.billm_gemm.argtypes = [vp, i64, i64, C.POINTER(BillmWeightsC), vp, i64, vp, vp]
@@ -142,8 +148,11 @@ def bwta_quantize_pack_acts(X: torch.Tensor, mode: int = TERNARY, thresh_ratio: 
 
 
 def bwta_gemm(a_mask, a_sign, a_scale, wbits, wscale, K: int, group: int = 0,
-              want_y: bool = True, want_dots: bool = False, status=None, out=None):
-    """Bit-packed GEMM. Returns (Y fp32 [M, N] or None, dots int32 [M, N] or None)."""
+              want_y: bool = True, want_dots: bool = False, status=None, out=None,
+              flags: int = 0):
+    """Bit-packed GEMM. Returns (Y fp32 [M, N] or None, dots int32 [M, N] or None).
+    flags=GEMM_WEIGHTS_READY (weights complete before the call) goes through
+    bwta_gemm_ex; 0 through bwta_gemm."""
     lib = _L()
     M, lda = a_mask.shape
     N, ldw = wbits.shape
@@ -152,10 +161,38 @@ def bwta_gemm(a_mask, a_sign, a_scale, wbits, wscale, K: int, group: int = 0,
         D = torch.empty((M, N), dtype=torch.int32, device=a_mask.device) if want_dots else None
     else:
         Y, D = out
-    _check("bwta_gemm", lib.bwta_gemm(
-        _ptr(a_mask), _ptr(a_sign), _ptr(a_scale), M, lda, _ptr(wbits), _ptr(wscale), N, ldw, K,
-        group, _ptr(Y), _row_stride(Y) if Y is not None else N, _ptr(D),
-        _row_stride(D) if D is not None else N, _ptr(status), _stream()))
+    ldY = _row_stride(Y) if Y is not None else N
+    ldD = _row_stride(D) if D is not None else N
+    if flags:
+        rc = lib.bwta_gemm_ex(_ptr(a_mask), _ptr(a_sign), _ptr(a_scale), M, lda, _ptr(wbits),
+                              _ptr(wscale), N, ldw, K, group, _ptr(Y), ldY, _ptr(D), ldD, flags,
+                              _ptr(status), _stream())
+        _check("bwta_gemm_ex", rc)
+    else:
+        _check("bwta_gemm", lib.bwta_gemm(
+            _ptr(a_mask), _ptr(a_sign), _ptr(a_scale), M, lda, _ptr(wbits), _ptr(wscale), N, ldw,
+            K, group, _ptr(Y), ldY, _ptr(D), ldD, _ptr(status), _stream()))
+    return Y, D
+
+
+def bwta_linear_decode(X, wbits, wscale, group: int = 0, mode: int = TERNARY,
+                       thresh_ratio: float = 0.5, want_y: bool = True, want_dots: bool = False,
+                       flags: int = 0, status=None, out=None):
+    """Fused decode: fp16 X [M<=8, K] -> ternarize in-kernel -> x packed weights.
+    Returns (Y fp32 [M, N] or None, dots int32 [M, N] or None)."""
+    lib = _L()
+    assert X.is_cuda and X.dtype == torch.float16 and X.dim() == 2 and X.stride(1) == 1
+    M, K = X.shape
+    N, ldw = wbits.shape
+    if out is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device) if want_y else None
+        D = torch.empty((M, N), dtype=torch.int32, device=X.device) if want_dots else None
+    else:
+        Y, D = out
+    _check("bwta_linear_decode", lib.bwta_linear_decode(
+        _ptr(X), M, K, _row_stride(X), mode, thresh_ratio, _ptr(wbits), _ptr(wscale), N, ldw, group,
+        _ptr(Y), _row_stride(Y) if Y is not None else N, _ptr(D),
+        _row_stride(D) if D is not None else N, flags, _ptr(status), _stream()))
     return Y, D
 
 

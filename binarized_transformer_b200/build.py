@@ -27,7 +27,7 @@ FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcomp
 
 LIB_SOURCES = ["pack.cu", "gemm.cu", "attn.cu", "billm.cu", "abi.cu"]
 MB_SOURCES = ["microbench.cu"]
-HEADERS = ["common.cuh", "tma.cuh"]
+HEADERS = ["common.cuh", "tma.cuh", "quant.cuh"]
 
 
 def _mtime(p):

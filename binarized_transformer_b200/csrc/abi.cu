@@ -63,6 +63,16 @@ int bwta_gemm(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_sca
               int64_t lda_words, const uint32_t *wbits, const float *wscale, int64_t N,
               int64_t ldw_words, int64_t K, int64_t group, float *Y, int64_t ldY, int32_t *dots,
               int64_t ldD, int32_t *d_status, bwta_stream_t stream) {
+  return bwta_gemm_ex(a_mask, a_sign, a_scale, M, lda_words, wbits, wscale, N, ldw_words, K, group,
+                      Y, ldY, dots, ldD, 0u, d_status, stream);
+}
+
+int bwta_gemm_ex(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_scale, int64_t M,
+                 int64_t lda_words, const uint32_t *wbits, const float *wscale, int64_t N,
+                 int64_t ldw_words, int64_t K, int64_t group, float *Y, int64_t ldY,
+                 int32_t *dots, int64_t ldD, uint32_t flags, int32_t *d_status,
+                 bwta_stream_t stream) {
+  if (flags & ~BWTA_GEMM_WEIGHTS_READY) return BWTA_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K <= 0) return BWTA_ERR_INVALID_ARG;
   if (K > BWTA_MAX_K) return BWTA_ERR_UNSUPPORTED;
   if (int r = check_group(group)) return r;
@@ -78,9 +88,32 @@ int bwta_gemm(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_sca
   cudaStream_t s = (cudaStream_t)stream;
   if (gemv_fits(M, lda_words, K, group))
     return cuda_status(launch_gemv(a_mask, a_sign, a_scale, M, lda_words, wbits, wscale, N,
-                                   ldw_words, K, group, Y, ldY, dots, ldD, s));
+                                   ldw_words, K, group, Y, ldY, dots, ldD,
+                                   (flags & BWTA_GEMM_WEIGHTS_READY) != 0, s));
   return cuda_status(launch_gemm_tiled(a_mask, a_sign, a_scale, M, lda_words, wbits, wscale, N,
                                        ldw_words, K, group, Y, ldY, dots, ldD, d_status, s));
+}
+
+int bwta_linear_decode(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
+                       float thresh_ratio, const uint32_t *wbits, const float *wscale, int64_t N,
+                       int64_t ldw_words, int64_t group, float *Y, int64_t ldY, int32_t *dots,
+                       int64_t ldD, uint32_t flags, int32_t *d_status, bwta_stream_t stream) {
+  if (flags & ~BWTA_GEMM_WEIGHTS_READY) return BWTA_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K <= 0 || ldX < K) return BWTA_ERR_INVALID_ARG;
+  if (mode != BWTA_TERNARY && mode != BWTA_BINARY) return BWTA_ERR_INVALID_ARG;
+  if (thresh_ratio != 0.5f) return BWTA_ERR_UNSUPPORTED;
+  if (M > 8 || !linear_decode_fits(M > 0 ? M : 1, K)) return BWTA_ERR_UNSUPPORTED;
+  if (int r = check_group(group)) return r;
+  if (!Y && !dots) return BWTA_ERR_INVALID_ARG;
+  if (Y && ldY < N) return BWTA_ERR_INVALID_ARG;
+  if (dots && ldD < N) return BWTA_ERR_INVALID_ARG;
+  if (M > 0 && !X) return BWTA_ERR_INVALID_ARG;
+  if (N > 0 && !wscale) return BWTA_ERR_INVALID_ARG;
+  if (int r = check_plane(wbits, N, ldw_words, K)) return r;
+  if (M == 0 || N == 0) return BWTA_OK;
+  return cuda_status(launch_linear_decode(X, M, K, ldX, mode, wbits, wscale, N, ldw_words, group,
+                                          Y, ldY, dots, ldD, (flags & BWTA_GEMM_WEIGHTS_READY) != 0,
+                                          d_status, (cudaStream_t)stream));
 }
 
 int bwta_attn_scores(const uint32_t *q_mask, const uint32_t *q_sign, const float *q_scale,
@@ -98,7 +131,7 @@ int bwta_attn_scores(const uint32_t *q_mask, const uint32_t *q_sign, const float
   if (S_f32 && BH * Lk > 0 && !k_scale) return BWTA_ERR_INVALID_ARG;
   if ((S_i32 && !aligned16(S_i32)) || (S_f32 && !aligned16(S_f32))) return BWTA_ERR_ALIGNMENT;
   return cuda_status(launch_attn_scores(q_mask, q_sign, q_scale, k_mask, k_sign, k_scale, BH, Lq,
-                                        Lk, ld_words, S_i32, S_f32, (cudaStream_t)stream));
+                                        Lk, D, ld_words, S_i32, S_f32, (cudaStream_t)stream));
 }
 
 static int check_billm(const billm_weights *W) {

@@ -7,34 +7,75 @@
 //     S = popc(mq & mk) - 2 * popc(mq & mk & (sq ^ sk))
 // The output (B*H*L*L scores) is far larger than the input (two planes of
 // D/32 words per row), so the kernel is bound by its output stream: each warp
-// writes 512 contiguous bytes per row with 16-byte streaming stores.
+// writes 512 contiguous bytes per row with 16-byte streaming stores, and the
+// small per-thread state keeps several CTAs (many stores in flight) per SM.
 #include "common.cuh"
 
 namespace bwta {
 
-constexpr int AT_TQ = 64, AT_TK = 128, AT_THREADS = 256;
+constexpr int AT_TQ = 128, AT_TK = 128, AT_THREADS = 256;
 
 __device__ __forceinline__ void st_cs(int32_t *p, int4 v) { __stcs(reinterpret_cast<int4 *>(p), v); }
 __device__ __forceinline__ void st_cs(float *p, float4 v) { __stcs(reinterpret_cast<float4 *>(p), v); }
 
-// CTA tile: 64 query rows x 128 key rows of one (batch, head). Warp w owns
-// query rows w + 8*r (r < 8); lane l owns key rows 4l .. 4l+3, so a warp's
-// stores for one query row are 128 consecutive scores.
-template <bool WI, bool WF, bool VEC>
-__global__ void __launch_bounds__(AT_THREADS)
+// Per word, with m = mq & mk and x = m & (sq ^ sk):
+//   popc(m) - 2*popc(x) = popc(m & ~x) - popc(x) = popc(agree) + popc(~x) - 32,
+// so a row pair's score is a plain sum of popcounts over 2*NW words minus 32*NW,
+// which carry-save adders fold into fewer POPCs (3 for NW = 2, 4 for NW = 4).
+__device__ __forceinline__ uint32_t agree_w(uint32_t m, uint32_t a, uint32_t b) {
+  uint32_t r;  // m & ~(a ^ b): 0xF0 & ~(0xCC ^ 0xAA) = 0x90
+  asm("lop3.b32 %0, %1, %2, %3, 0x90;" : "=r"(r) : "r"(m), "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t ndis_w(uint32_t m, uint32_t a, uint32_t b) {
+  uint32_t r;  // ~(m & (a ^ b)): ~0x60 = 0x9F
+  asm("lop3.b32 %0, %1, %2, %3, 0x9F;" : "=r"(r) : "r"(m), "r"(a), "r"(b));
+  return r;
+}
+
+template <int NW>
+__device__ __forceinline__ int tern_dot(const uint4 &qm, const uint4 &qs, const uint4 &km, const uint4 &ks) {
+  const uint32_t m0 = qm.x & km.x;
+  if (NW == 1) return __popc(agree_w(m0, qs.x, ks.x)) - __popc(lop3_and_xor(m0, qs.x, ks.x));
+  const uint32_t m1 = qm.y & km.y;
+  if (NW == 2)
+    return popc4_csa(agree_w(m0, qs.x, ks.x), agree_w(m1, qs.y, ks.y), ndis_w(m0, qs.x, ks.x),
+                     ndis_w(m1, qs.y, ks.y)) - 64;
+  const uint32_t m2 = qm.z & km.z, m3 = qm.w & km.w;
+  const uint32_t a0 = agree_w(m0, qs.x, ks.x), a1 = agree_w(m1, qs.y, ks.y),
+                 a2 = agree_w(m2, qs.z, ks.z), a3 = agree_w(m3, qs.w, ks.w);
+  const uint32_t n0 = ndis_w(m0, qs.x, ks.x), n1 = ndis_w(m1, qs.y, ks.y),
+                 n2 = ndis_w(m2, qs.z, ks.z), n3 = ndis_w(m3, qs.w, ks.w);
+  // eight words -> ones (s3, n3), twos (s4), fours (c4)
+  const uint32_t s1 = xor3(a0, a1, a2), c1 = maj3(a0, a1, a2);
+  const uint32_t s2 = xor3(a3, n0, n1), c2 = maj3(a3, n0, n1);
+  const uint32_t s3 = xor3(s1, s2, n2), c3 = maj3(s1, s2, n2);
+  const uint32_t s4 = xor3(c1, c2, c3), c4 = maj3(c1, c2, c3);
+  return __popc(s3) + __popc(n3) + 2 * __popc(s4) + 4 * __popc(c4) - 128;
+}
+
+// CTA tile: 128 query rows x 128 key rows of one (batch, head). Lane l holds
+// the planes of key rows 4l .. 4l+3 in registers for the whole tile; warp w
+// walks query rows w, w + 8, ... (16 of them), and for each computes its 4
+// scores and stores them at once (16 bytes; 512 contiguous bytes per warp), so
+// no scores are held in registers and many CTAs stay resident per SM. NW =
+// data words per row (1 or 2 in one chunk; 4 = any D in 4-word chunks).
+template <int NW, bool WI, bool WF, bool VEC>
+__global__ void __launch_bounds__(AT_THREADS, 4)
 k_attn_scores(const uint32_t *__restrict__ qm, const uint32_t *__restrict__ qs,
               const float *__restrict__ qscale, const uint32_t *__restrict__ km,
               const uint32_t *__restrict__ ks, const float *__restrict__ kscale, int64_t Lq,
               int64_t Lk, int ld, int32_t *__restrict__ Si, float *__restrict__ Sf) {
   extern __shared__ uint4 at_sm[];
-  const int nc = ld / 4;  // 4-word chunks per row
+  const int nc = NW == 4 ? ld / 4 : 1;  // 4-word chunks per row
   uint4 *sQm = at_sm;
   uint4 *sQs = sQm + AT_TQ * nc;
   uint4 *sKm = sQs + AT_TQ * nc;
   uint4 *sKs = sKm + AT_TK * nc;
   float *sq = reinterpret_cast<float *>(sKs + AT_TK * nc);
   float *sk = sq + AT_TQ;
-
+  pdl_trigger();
+  pdl_wait();
   const int64_t bh = blockIdx.z;
   const int64_t i0 = (int64_t)blockIdx.y * AT_TQ, j0 = (int64_t)blockIdx.x * AT_TK;
   const uint4 z4 = make_uint4(0, 0, 0, 0);
@@ -63,45 +104,40 @@ k_attn_scores(const uint32_t *__restrict__ qm, const uint32_t *__restrict__ qs,
   __syncthreads();
 
   const int w = threadIdx.x / 32, l = threadIdx.x % 32;
-  int P[8][4], X[8][4];
+  const int64_t jb = j0 + 4 * l;
+  float skv[4];
 #pragma unroll
-  for (int r = 0; r < 8; ++r)
-#pragma unroll
-    for (int t = 0; t < 4; ++t) P[r][t] = X[r][t] = 0;
-
-  for (int c = 0; c < nc; ++c) {
-    uint4 kmv[4], ksv[4];
+  for (int t = 0; t < 4; ++t) skv[t] = WF ? sk[4 * l + t] : 0.0f;
+  uint4 kmv[4], ksv[4];
+  if (NW != 4) {
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      kmv[t] = sKm[(4 * l + t) * nc + c];
-      ksv[t] = sKs[(4 * l + t) * nc + c];
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const uint4 a = sQm[(w + 8 * r) * nc + c], b = sQs[(w + 8 * r) * nc + c];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const uint32_t m0 = a.x & kmv[t].x, m1 = a.y & kmv[t].y, m2 = a.z & kmv[t].z,
-                       m3 = a.w & kmv[t].w;
-        P[r][t] += __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
-        X[r][t] += __popc(lop3_and_xor(m0, b.x, ksv[t].x)) + __popc(lop3_and_xor(m1, b.y, ksv[t].y)) +
-                   __popc(lop3_and_xor(m2, b.z, ksv[t].z)) + __popc(lop3_and_xor(m3, b.w, ksv[t].w));
-      }
+      kmv[t] = sKm[4 * l + t];
+      ksv[t] = sKs[4 * l + t];
     }
   }
-
+  for (int r = w; r < AT_TQ; r += AT_THREADS / 32) {
+    const int64_t i = i0 + r;
+    if (i >= Lq) break;
+    int d[4] = {0, 0, 0, 0};
+    if (NW != 4) {
+      const uint4 a = sQm[r], b = sQs[r];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int64_t i = i0 + w + 8 * r;
-    if (i >= Lq) continue;
-    const int64_t jb = j0 + 4 * l;
+      for (int t = 0; t < 4; ++t) d[t] = tern_dot<NW>(a, b, kmv[t], ksv[t]);
+    } else {
+      for (int c = 0; c < nc; ++c) {
+        const uint4 a = sQm[r * nc + c], b = sQs[r * nc + c];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          d[t] += tern_dot<4>(a, b, sKm[(4 * l + t) * nc + c], sKs[(4 * l + t) * nc + c]);
+      }
+    }
     const int64_t o = (bh * Lq + i) * Lk + jb;
-    int d[4];
     float f[4];
+    if (WF) {
+      const float sqi = sq[r];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      d[t] = P[r][t] - 2 * X[r][t];
-      if (WF) f[t] = (__int2float_rn(d[t]) * sq[w + 8 * r]) * sk[4 * l + t];
+      for (int t = 0; t < 4; ++t) f[t] = (__int2float_rn(d[t]) * sqi) * skv[t];
     }
     if (VEC && jb + 3 < Lk) {
       if (WI) st_cs(Si + o, make_int4(d[0], d[1], d[2], d[3]));
@@ -117,37 +153,50 @@ k_attn_scores(const uint32_t *__restrict__ qm, const uint32_t *__restrict__ qs,
   }
 }
 
-template <bool WI, bool WF, bool VEC>
+template <int NW, bool WI, bool WF, bool VEC>
 static cudaError_t launch_attn_t(const uint32_t *qm, const uint32_t *qs, const float *qscale,
                                  const uint32_t *km, const uint32_t *ks, const float *kscale,
                                  int64_t BH, int64_t Lq, int64_t Lk, int64_t ld, int32_t *Si,
                                  float *Sf, cudaStream_t s) {
-  const int nc = (int)(ld / 4);
+  const int nc = NW == 4 ? (int)(ld / 4) : 1;
   const size_t smem = (size_t)(AT_TQ + AT_TK) * nc * 2 * 16 + (AT_TQ + AT_TK) * 4;
-  auto kern = k_attn_scores<WI, WF, VEC>;
+  auto kern = k_attn_scores<NW, WI, WF, VEC>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   dim3 grid((unsigned)ceil_div<int64_t>(Lk, AT_TK), (unsigned)ceil_div<int64_t>(Lq, AT_TQ),
             (unsigned)BH);
-  kern<<<grid, AT_THREADS, smem, s>>>(qm, qs, qscale, km, ks, kscale, Lq, Lk, (int)ld, Si, Sf);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(AT_THREADS), smem, s, qm, qs, qscale, km, ks, kscale, Lq, Lk,
+                    (int)ld, Si, Sf);
 }
 
-cudaError_t launch_attn_scores(const uint32_t *qm, const uint32_t *qs, const float *qscale,
-                               const uint32_t *km, const uint32_t *ks, const float *kscale,
-                               int64_t BH, int64_t Lq, int64_t Lk, int64_t ld, int32_t *Si,
-                               float *Sf, cudaStream_t s) {
-  if (BH == 0 || Lq == 0 || Lk == 0) return cudaSuccess;
+template <int NW>
+static cudaError_t launch_attn_nw(const uint32_t *qm, const uint32_t *qs, const float *qscale,
+                                  const uint32_t *km, const uint32_t *ks, const float *kscale,
+                                  int64_t BH, int64_t Lq, int64_t Lk, int64_t ld, int32_t *Si,
+                                  float *Sf, cudaStream_t s) {
   const bool vec = (Lk % 4) == 0;
-#define BWTA_AT(WI, WF)                                                                           \
-  return vec ? launch_attn_t<WI, WF, true>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, Si, Sf, s) \
-             : launch_attn_t<WI, WF, false>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, Si, Sf, s)
+#define BWTA_AT(WI, WF)                                                                         \
+  return vec ? launch_attn_t<NW, WI, WF, true>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, Si, \
+                                               Sf, s)                                            \
+             : launch_attn_t<NW, WI, WF, false>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, Si, \
+                                                Sf, s)
   if (Si && Sf) BWTA_AT(true, true);
   if (Si) BWTA_AT(true, false);
   BWTA_AT(false, true);
 #undef BWTA_AT
+}
+
+cudaError_t launch_attn_scores(const uint32_t *qm, const uint32_t *qs, const float *qscale,
+                               const uint32_t *km, const uint32_t *ks, const float *kscale,
+                               int64_t BH, int64_t Lq, int64_t Lk, int64_t D, int64_t ld,
+                               int32_t *Si, float *Sf, cudaStream_t s) {
+  if (BH == 0 || Lq == 0 || Lk == 0) return cudaSuccess;
+  const int64_t nw = ceil_div<int64_t>(D, 32);  // data words per row
+  if (nw == 1) return launch_attn_nw<1>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, Si, Sf, s);
+  if (nw == 2) return launch_attn_nw<2>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, Si, Sf, s);
+  return launch_attn_nw<4>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, Si, Sf, s);
 }
 
 }  // namespace bwta

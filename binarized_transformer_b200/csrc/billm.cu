@@ -26,6 +26,8 @@ k_billm_salient(const float *__restrict__ W, int64_t N, int64_t ldW, int n_sal,
                 uint8_t *__restrict__ sal, int32_t *d_status) {
   __shared__ double metric[128];
   __shared__ unsigned char taken[128];
+  pdl_trigger();
+  pdl_wait();
   const int c = threadIdx.x;
   const int64_t col = (int64_t)blockIdx.x * 128 + c;
   double acc = 0.0;
@@ -74,6 +76,8 @@ k_billm_quantize(const float *__restrict__ W, int64_t N, int64_t K, int64_t ldW,
                  int split, const uint8_t *__restrict__ sal, uint32_t *__restrict__ sign,
                  uint32_t *__restrict__ gmap, int64_t ldw, uint8_t *__restrict__ res,
                  float *__restrict__ bscale) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t nb = K / 128;
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= N * nb) return;
@@ -140,15 +144,14 @@ cudaError_t launch_billm_pack(const float *W, int64_t ldW, int split, const bill
   const int64_t N = o->N, K = o->K, nb = K / 128;
   if (N == 0) return cudaSuccess;
   uint8_t *sal = const_cast<uint8_t *>(o->sal);
-  k_billm_salient<<<(unsigned)nb, 128, 0, s>>>(W, N, ldW, (int)o->n_sal, sal, d_status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(k_billm_salient, dim3((unsigned)nb), dim3(128), 0, s, W, N, ldW,
+                             (int)o->n_sal, sal, d_status);
   if (e != cudaSuccess) return e;
   const int64_t total = N * nb;
-  k_billm_quantize<<<(unsigned)ceil_div<int64_t>(total, 256), 256, 0, s>>>(
-      W, N, K, ldW, (int)o->n_sal, split, sal, const_cast<uint32_t *>(o->sign),
-      const_cast<uint32_t *>(o->gmap), o->ldw_words, const_cast<uint8_t *>(o->res),
-      const_cast<float *>(o->bscale));
-  return cudaGetLastError();
+  return launch_pdl(k_billm_quantize, dim3((unsigned)ceil_div<int64_t>(total, 256)), dim3(256), 0, s,
+                    W, N, K, ldW, (int)o->n_sal, split, (const uint8_t *)sal,
+                    const_cast<uint32_t *>(o->sign), const_cast<uint32_t *>(o->gmap), o->ldw_words,
+                    const_cast<uint8_t *>(o->res), const_cast<float *>(o->bscale));
 }
 
 // ================================================================= GEMM
@@ -172,6 +175,8 @@ k_billm_gemm(const uint16_t *__restrict__ X, int64_t M, int64_t ldX, const uint3
              int64_t K, int64_t ldw, int n_sal, float *__restrict__ Y, int64_t ldY,
              int32_t *d_status) {
   extern __shared__ float xs[];  // [MT][128][nb]
+  pdl_trigger();
+  pdl_wait();
   const int nb = (int)(K / 128);
   uint8_t *ssal = reinterpret_cast<uint8_t *>(xs + (size_t)MT * K);
   for (int i = threadIdx.x; i < nb * n_sal; i += BG_THREADS) ssal[i] = sal[i];
@@ -272,10 +277,9 @@ static cudaError_t launch_bg_t(const uint16_t *X, int64_t M, int64_t ldX, const 
   if (attr != cudaSuccess) return attr;
   const size_t smem = (size_t)MT * W->K * 4 + 8 * (W->K / 128);
   const int64_t blocks = std::min<int64_t>(ceil_div<int64_t>(W->N, BG_WARPS), 148);
-  kern<<<(unsigned)blocks, BG_THREADS, smem, s>>>(X, M, ldX, W->sign, W->gmap, W->res, W->sal,
-                                                  W->bscale, W->N, W->K, W->ldw_words,
-                                                  (int)W->n_sal, Y, ldY, d_status);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3((unsigned)blocks), dim3(BG_THREADS), smem, s, X, M, ldX, W->sign,
+                    W->gmap, W->res, W->sal, W->bscale, W->N, W->K, W->ldw_words, (int)W->n_sal, Y,
+                    ldY, d_status);
 }
 
 cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,

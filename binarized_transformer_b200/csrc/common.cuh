@@ -43,12 +43,67 @@ __device__ __forceinline__ uint32_t lop3_and_xor(uint32_t m, uint32_t a, uint32_
   return r;
 }
 
+// Full adder on 32 bit positions at once: per bit, a + b + c = sum + 2*carry.
+__device__ __forceinline__ uint32_t xor3(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;  // 0xF0 ^ 0xCC ^ 0xAA = 0x96
+  asm("lop3.b32 %0, %1, %2, %3, 0x96;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t maj3(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;  // majority of (0xF0, 0xCC, 0xAA) = 0xE8
+  asm("lop3.b32 %0, %1, %2, %3, 0xE8;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+// popc(t0) + popc(t1) + popc(t2) + popc(t3) with three POPCs: a carry-save
+// full adder folds t0, t1, t2 into a sum plane (weight 1) and a carry plane
+// (weight 2). Four words take at least three POPCs (0..4 per bit needs three
+// bit planes); the two extra LOP3s run on the ALU pipe, which has 4x the
+// POPC pipe's throughput.
+__device__ __forceinline__ int popc4_csa(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3) {
+  return __popc(xor3(t0, t1, t2)) + __popc(t3) + 2 * __popc(maj3(t0, t1, t2));
+}
+
 // (float)d for |d| < 2^22 via the 1.5*2^23 bias trick: exact, and it keeps
 // the conversion off the int->float conversion unit. `biased` = d + 0x4B400000.
 __device__ __forceinline__ float biased_int_to_float(int32_t biased) {
   return __int_as_float(biased) - 12582912.0f;
 }
 constexpr int32_t INT_FLOAT_BIAS = 0x4B400000;
+
+// Programmatic dependent launch. Every kernel lets the next kernel in the
+// stream be scheduled as soon as all of its own blocks are running, and waits
+// for the previous kernel's completion (and memory) before it reads any global
+// input. Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+#ifndef __CUDACC_RTC__
+// Launch `kern` on `s` with programmatic stream serialization allowed.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+#ifdef BWTA_NO_PDL
+  cfg.numAttrs = 0;  // build-time option: plain stream-ordered launches
+#else
+  cfg.numAttrs = 1;
+#endif
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+#endif
 
 template <typename T>
 __host__ __device__ __forceinline__ T ceil_div(T a, T b) {
@@ -72,12 +127,17 @@ cudaError_t launch_gemm_tiled(const uint32_t *am, const uint32_t *as, const floa
 cudaError_t launch_gemv(const uint32_t *am, const uint32_t *as, const float *ascale, int64_t M,
                         int64_t lda, const uint32_t *wb, const float *wscale, int64_t N,
                         int64_t ldw, int64_t K, int64_t group, float *Y, int64_t ldY,
-                        int32_t *dots, int64_t ldD, cudaStream_t s);
+                        int32_t *dots, int64_t ldD, bool weights_ready, cudaStream_t s);
 bool gemv_fits(int64_t M, int64_t lda, int64_t K, int64_t group);
+bool linear_decode_fits(int64_t M, int64_t K);
+cudaError_t launch_linear_decode(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
+                                 const uint32_t *wb, const float *wscale, int64_t N, int64_t ldw,
+                                 int64_t group, float *Y, int64_t ldY, int32_t *dots, int64_t ldD,
+                                 bool ready, int32_t *d_status, cudaStream_t s);
 cudaError_t launch_attn_scores(const uint32_t *qm, const uint32_t *qs, const float *qscale,
                                const uint32_t *km, const uint32_t *ks, const float *kscale,
-                               int64_t BH, int64_t Lq, int64_t Lk, int64_t ld, int32_t *Si,
-                               float *Sf, cudaStream_t s);
+                               int64_t BH, int64_t Lq, int64_t Lk, int64_t D, int64_t ld,
+                               int32_t *Si, float *Sf, cudaStream_t s);
 cudaError_t launch_billm_pack(const float *W, int64_t ldW, int split, const billm_weights *out,
                               int32_t *d_status, cudaStream_t s);
 cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,

@@ -5,6 +5,7 @@
 // Co-design -- abstract: binary weights, activations ternarized by projecting
 // tiny values to zero; Figure 6: 32 fp16 values packed into one 32-bit word.
 #include "common.cuh"
+#include "quant.cuh"
 
 namespace bwta {
 
@@ -22,6 +23,8 @@ k_pack_weights(const float *__restrict__ W, int64_t N, int64_t K, int64_t ldW, i
                int64_t G, uint32_t *__restrict__ wbits, int64_t ldw,
                float *__restrict__ wscale, int32_t *d_status) {
   __shared__ float tile[PW_WARPS][32][33];
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t row0 = ((int64_t)blockIdx.x * PW_WARPS + warp) * 32;
   if (row0 >= N) return;
@@ -79,9 +82,8 @@ cudaError_t launch_pack_weights(const float *W, int64_t N, int64_t K, int64_t ld
   const int64_t G = ceil_div(K, gs);
   const int64_t warps = ceil_div<int64_t>(N, 32);
   const int64_t blocks = ceil_div<int64_t>(warps, PW_WARPS);
-  k_pack_weights<<<(unsigned)blocks, PW_WARPS * 32, 0, s>>>(W, N, K, ldW, gs, G, wbits, ldw,
-                                                            wscale, d_status);
-  return cudaGetLastError();
+  return launch_pdl(k_pack_weights, dim3((unsigned)blocks), dim3(PW_WARPS * 32), 0, s, W, N, K, ldW,
+                    gs, G, wbits, ldw, wscale, d_status);
 }
 
 // ======================================================== activations (K1)
@@ -98,98 +100,6 @@ cudaError_t launch_pack_weights(const float *W, int64_t N, int64_t K, int64_t ld
 //          the same IEEE roundings as the definition (int64->fp64, fp64
 //          divide, times 2^-24, fp64->fp32).
 // The row stays in registers between the passes for rows up to 16 steps.
-constexpr int QA_THREADS = 256;
-constexpr int QA_NREG = 8;
-
-template <int T>
-__device__ __forceinline__ uint64_t team_sum_u64(uint64_t v, uint64_t *red) {
-  if constexpr (T <= 32) {
-#pragma unroll
-    for (int o = T / 2; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-    return v;
-  } else {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-    const int warp = threadIdx.x / 32;
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[warp] = v;
-    __syncthreads();
-    const int w0 = (threadIdx.x / T) * (T / 32);
-    uint64_t r = 0;
-#pragma unroll
-    for (int i = 0; i < T / 32; ++i) r += red[w0 + i];
-    return r;
-  }
-}
-
-// 8 halves starting at k0 (zeros past K). VEC: the row start is 16-byte
-// aligned (X aligned, ldX % 8 == 0), so full groups use one 16-byte load.
-template <bool VEC>
-__device__ __forceinline__ uint4 load_half8(const uint16_t *row, int64_t k0, int64_t K, bool valid) {
-  if (!valid || k0 >= K) return make_uint4(0, 0, 0, 0);
-  if (VEC && k0 + 8 <= K) return __ldg(reinterpret_cast<const uint4 *>(row + k0));
-  uint32_t w[4] = {0, 0, 0, 0};
-  for (int i = 0; i < 8; ++i)
-    if (k0 + i < K) w[i >> 1] |= (uint32_t)__ldg(row + k0 + i) << (16 * (i & 1));
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-__device__ __forceinline__ uint64_t sum_mag8(const uint4 &v, bool &bad) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint64_t s = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t hm = (w[i >> 1] >> (16 * (i & 1))) & 0x7FFFu;
-    bad |= hm >= 0x7C00u;
-    s += mag_units(hm);
-  }
-  return s;
-}
-
-// keep / sign bit patterns of 8 halves, plus the sum of the kept magnitudes.
-template <bool TERNARY>
-__device__ __forceinline__ void keep8(const uint4 &v, uint32_t hT, int64_t k0, int64_t K,
-                                      uint32_t &kb, uint32_t &sb, uint64_t &ks) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  kb = 0;
-  sb = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t h = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
-    const uint32_t hm = h & 0x7FFFu;
-    uint32_t keep;
-    if (TERNARY) {
-      keep = hm > hT;
-      if (keep) ks += mag_units(hm);
-    } else {
-      keep = (k0 + i) < K;
-    }
-    const uint32_t neg = keep & (h >> 15) & (hm != 0u);
-    kb |= keep << i;
-    sb |= neg << i;
-  }
-}
-
-// Merge the 8-bit patterns of a 16-lane chunk group into 4 words; lane 0 of
-// the group stores them (one 128-bit store per plane).
-__device__ __forceinline__ void store_chunk(uint32_t kb, uint32_t sb, uint32_t *mrow,
-                                            uint32_t *srow, int chunk, bool do_store) {
-  const int l16 = threadIdx.x & 15;
-  uint32_t mw = kb << (8 * (l16 & 3)), sw = sb << (8 * (l16 & 3));
-  mw |= __shfl_xor_sync(FULL, mw, 1);
-  sw |= __shfl_xor_sync(FULL, sw, 1);
-  mw |= __shfl_xor_sync(FULL, mw, 2);
-  sw |= __shfl_xor_sync(FULL, sw, 2);
-  const uint32_t m1 = __shfl_down_sync(FULL, mw, 4), m2 = __shfl_down_sync(FULL, mw, 8),
-                 m3 = __shfl_down_sync(FULL, mw, 12);
-  const uint32_t s1 = __shfl_down_sync(FULL, sw, 4), s2 = __shfl_down_sync(FULL, sw, 8),
-                 s3 = __shfl_down_sync(FULL, sw, 12);
-  if (do_store && l16 == 0) {
-    *reinterpret_cast<uint4 *>(mrow + 4 * chunk) = make_uint4(mw, m1, m2, m3);
-    *reinterpret_cast<uint4 *>(srow + 4 * chunk) = make_uint4(sw, s1, s2, s3);
-  }
-}
-
 template <int T, bool TERNARY, bool VEC>
 __global__ void __launch_bounds__(QA_THREADS)
 k_quantize_pack_acts(const uint16_t *__restrict__ X, int64_t M, int64_t K, int64_t ldX,
@@ -198,6 +108,8 @@ k_quantize_pack_acts(const uint16_t *__restrict__ X, int64_t M, int64_t K, int64
   constexpr int TEAMS = QA_THREADS / T;
   constexpr int CPS = T / 16;  // chunks per step
   __shared__ uint64_t red[QA_THREADS / 32];
+  pdl_trigger();
+  pdl_wait();
   const int t = threadIdx.x % T;
   const int64_t row = (int64_t)blockIdx.x * TEAMS + threadIdx.x / T;
   const bool valid = row < M;
@@ -277,18 +189,16 @@ static cudaError_t launch_qa_t(const uint16_t *X, int64_t M, int64_t K, int64_t 
   constexpr int TEAMS = QA_THREADS / T;
   const int64_t blocks = ceil_div<int64_t>(M, TEAMS);
   const bool vec = (reinterpret_cast<uintptr_t>(X) & 15u) == 0 && ldX % 8 == 0;
-#define BWTA_QA(TER, V)                                                                        \
-  k_quantize_pack_acts<T, TER, V><<<(unsigned)blocks, QA_THREADS, 0, s>>>(X, M, K, ldX, mask, \
-                                                                          sign, lda, scale, d_status)
+#define BWTA_QA(TER, V)                                                                          \
+  return launch_pdl(k_quantize_pack_acts<T, TER, V>, dim3((unsigned)blocks), dim3(QA_THREADS), 0, s, \
+                    X, M, K, ldX, mask, sign, lda, scale, d_status)
   if (mode == BWTA_TERNARY) {
     if (vec) BWTA_QA(true, true);
-    else BWTA_QA(true, false);
-  } else {
-    if (vec) BWTA_QA(false, true);
-    else BWTA_QA(false, false);
+    BWTA_QA(true, false);
   }
+  if (vec) BWTA_QA(false, true);
+  BWTA_QA(false, false);
 #undef BWTA_QA
-  return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_pack_acts(const uint16_t *X, int64_t M, int64_t K, int64_t ldX,

@@ -119,6 +119,39 @@ int bwta_gemm(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_sca
               int64_t ldw_words, int64_t K, int64_t group, float *Y, int64_t ldY, int32_t *dots,
               int64_t ldD, int32_t *d_status, bwta_stream_t stream);
 
+/* bwta_gemm with flags. BWTA_GEMM_WEIGHTS_READY promises that `wbits` and
+ * `wscale` were complete before this call was enqueued (e.g. packed at load
+ * time, then the stream or device was synchronized). The kernels launch with
+ * programmatic dependent launch: without the flag they read nothing before
+ * the previous kernel in the stream has completed; with it the decode GEMV
+ * starts streaming the weights while the previous kernel (typically the
+ * activation packer) is still running, and waits only before it reads the
+ * activation planes. Passing the flag for weights that a still-running kernel
+ * writes is a race. Other flags bits must be 0. */
+#define BWTA_GEMM_WEIGHTS_READY 0x1u
+int bwta_gemm_ex(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_scale, int64_t M,
+                 int64_t lda_words, const uint32_t *wbits, const float *wscale, int64_t N,
+                 int64_t ldw_words, int64_t K, int64_t group, float *Y, int64_t ldY,
+                 int32_t *dots, int64_t ldD, uint32_t flags, int32_t *d_status,
+                 bwta_stream_t stream);
+
+/* Decode linear layer in one kernel: ternarize (or binarize) M <= 8 fp16 rows
+ * and multiply them by packed binary weights, without writing the activation
+ * planes to memory (BWTA abstract: ternary activations; bit-packed MatMul).
+ * Equivalent to bwta_quantize_pack_acts followed by bwta_gemm: the same planes
+ * and scales bit for bit, the same integer dots; fp32 outputs within the
+ * tolerance of the decode GEMV (group terms summed as a tree).
+ *  X          fp16 bits [M][ldX], any alignment
+ *  mode, thresh_ratio   as bwta_quantize_pack_acts
+ *  wbits, wscale, N, ldw_words, group, Y, ldY, dots, ldD   as bwta_gemm
+ *  flags      0 or BWTA_GEMM_WEIGHTS_READY (see bwta_gemm_ex)
+ *  Limits: M <= 8, ceil(K/128) <= 128 (K <= 16384); else UNSUPPORTED.
+ *  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; NONFINITE flag. */
+int bwta_linear_decode(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
+                       float thresh_ratio, const uint32_t *wbits, const float *wscale, int64_t N,
+                       int64_t ldw_words, int64_t group, float *Y, int64_t ldY, int32_t *dots,
+                       int64_t ldD, uint32_t flags, int32_t *d_status, bwta_stream_t stream);
+
 /* Ternary attention scores Q . K^T per batch*head (BWTA abstract: binary /
  * ternary MatMul for the attention operators). Both operands come from
  * bwta_quantize_pack_acts over rows of length D.

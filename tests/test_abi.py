@@ -78,6 +78,9 @@ def test_validation_rejects_before_launch(lib):
         E.BWTA_ERR_INVALID_ARG
     assert g(MISALIGNED, FAKE, FAKE, 4, 4, FAKE, FAKE, 4, 4, 64, 0, FAKE, 4, None, 4, None, None) == \
         E.BWTA_ERR_ALIGNMENT
+    gx = lib.bwta_gemm_ex
+    assert gx(FAKE, FAKE, FAKE, 4, 4, FAKE, FAKE, 4, 4, 64, 0, FAKE, 4, None, 4, 2, None, None) == \
+        E.BWTA_ERR_INVALID_ARG
     # bwta_attn_scores: no outputs, ld too large
     at = lib.bwta_attn_scores
     assert at(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 4, 64, 4, None, None, None) == E.BWTA_ERR_INVALID_ARG

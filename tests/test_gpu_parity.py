@@ -174,6 +174,65 @@ def test_gemv_small(M, N, K, group):
     run_linear(X, W, group)
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (1, 300, 11008), (3, 1000, 4096)])
+def test_gemv_weights_ready_flag(M, N, K):
+    """bwta_gemm_ex(WEIGHTS_READY): weights packed and synchronized first, then
+    the GEMV streams them before waiting on the activation packer."""
+    X = workloads.edge_acts(M, K, "student", tag=N)
+    W = workloads.edge_weights(N, K, tag=N)
+    wb, ws = gpu_pack_weights(W, 128)
+    torch.cuda.synchronize()
+    ref = oracle.linear(X, W, 128)
+    Xd = dev(X)
+    for _ in range(2):
+        m, s, sc = bt.bwta_quantize_pack_acts(Xd)
+        Y, D = bt.bwta_gemm(m, s, sc, wb, ws, K, 128, want_dots=True, flags=bt.GEMM_WEIGHTS_READY)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(D.cpu().numpy(), ref["dots"])
+        assert_close_rel(Y.cpu().numpy(), ref["yref"], ref["mag"], what="gemv ready")
+
+
+@pytest.mark.parametrize("ready", [False, True])
+@pytest.mark.parametrize("M", [1, 3, 8])
+@pytest.mark.parametrize("N,K,group", [(100, 256, 0), (64, 4096, 128), (50, 11008, 128),
+                                       (33, 300, 128), (40, 16384, 0)])
+def test_linear_decode_fused(M, N, K, group, ready):
+    """bwta_linear_decode ternarizes inside the kernel: same dots as the
+    two-call path (exact), fp32 within tolerance."""
+    X = workloads.edge_acts(M, K, "student", tag=7 * N + M)
+    W = workloads.edge_weights(N, K, tag=N + M)
+    wb, ws = gpu_pack_weights(W, group)
+    torch.cuda.synchronize()
+    ref = oracle.linear(X, W, group)
+    Yv, ycheck = guarded((M, N), torch.float32)
+    Dv, dcheck = guarded((M, N), torch.int32)
+    st = bt.new_status()
+    bt.bwta_linear_decode(dev(X), wb, ws, group, want_dots=True, status=st, out=(Yv, Dv),
+                          flags=bt.GEMM_WEIGHTS_READY if ready else 0)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    ycheck()
+    dcheck()
+    np.testing.assert_array_equal(Dv.cpu().numpy(), ref["dots"])
+    assert_close_rel(Yv.cpu().numpy(), ref["yref"], ref["mag"] if group else None, what="decode")
+
+
+def test_linear_decode_binary_and_zero_rows():
+    K, N = 512, 64
+    W = workloads.edge_weights(N, K, tag=5)
+    wb, ws = gpu_pack_weights(W, 128)
+    X = workloads.edge_acts(4, K, "normal", tag=5)
+    X[1] = 0
+    for mode, ternary in ((bt.BINARY, False), (bt.TERNARY, True)):
+        Y, D = bt.bwta_linear_decode(dev(X), wb, ws, 128, mode=mode, want_dots=True)
+        a, sc = oracle.quantize_acts(X, ternary=ternary)
+        b, alpha = oracle.binarize_weights(W, 128)
+        d = oracle.int_dots(a, b, 128)
+        yref, mag, _ = oracle.linear_out(d, alpha, sc)
+        np.testing.assert_array_equal(D.cpu().numpy(), d.sum(axis=2))
+        assert_close_rel(Y.cpu().numpy(), yref, mag, what="decode binary")
+
+
 def test_gemm_tiny_workload():
     t = workloads.tiny()
     Y, yrep = run_linear(t["X"], t["W"], 0)
