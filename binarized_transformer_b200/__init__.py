@@ -25,7 +25,8 @@ STATUS_NONFINITE, STATUS_TIMEOUT = 0x1, 0x2
 TERNARY, BINARY = 0, 1
 ERROR_NAMES = {1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA"}
 
-EXPORTS = ["bwta_pack_weights", "bwta_quantize_pack_acts", "bwta_gemm", "bwta_gemm_ex",
+EXPORTS = ["bwta_pack_weights", "bwta_quantize_pack_acts", "bwta_quantize_pack_acts_ex",
+           "bwta_gemm", "bwta_gemm_ex", "bwta_gemm_tc",
            "bwta_linear_decode", "bwta_attn_scores", "billm_pack_weights", "billm_gemm",
            "bwta_version"]
 GEMM_WEIGHTS_READY = 0x1
@@ -58,6 +59,10 @@ def load_library(path: str = LIB_PATH):
     vp, i64, ci, cf = C.c_void_p, C.c_int64, C.c_int, C.c_float
     lib.bwta_pack_weights.argtypes = [vp, i64, i64, i64, i64, vp, i64, vp, vp, vp]
     lib.bwta_quantize_pack_acts.argtypes = [vp, i64, i64, i64, ci, cf, vp, vp, i64, vp, vp, vp]
+    lib.bwta_quantize_pack_acts_ex.argtypes = [vp, i64, i64, i64, ci, cf, vp, vp, i64, vp, i64, vp,
+                                               vp, vp]
+    lib.bwta_gemm_tc.argtypes = [vp, i64, vp, i64, vp, vp, i64, i64, i64, i64, vp, i64, vp, i64,
+                                 vp, vp]
     lib.bwta_gemm.argtypes = [vp, vp, vp, i64, i64, vp, vp, i64, i64, i64, i64, vp, i64, vp, i64,
                               vp, vp]
     lib.bwta_gemm_ex.argtypes = [vp, vp, vp, i64, i64, vp, vp, i64, i64, i64, i64, vp, i64, vp,
@@ -145,6 +150,49 @@ def bwta_quantize_pack_acts(X: torch.Tensor, mode: int = TERNARY, thresh_ratio: 
         _ptr(X), M, K, _row_stride(X), mode, thresh_ratio, _ptr(mask), _ptr(sign), ld, _ptr(scale),
         _ptr(status), _stream()))
     return mask, sign, scale
+
+
+def e4m3_ld_for(K: int) -> int:
+    """Row stride in bytes of E4M3 activations for the tensor-core GEMM."""
+    return ld_words_for(K) * 32
+
+
+def bwta_quantize_pack_acts_ex(X: torch.Tensor, mode: int = TERNARY, thresh_ratio: float = 0.5,
+                               planes: bool = True, e4m3: bool = True, status=None, out=None):
+    """fp16 X [M, K] -> (mask, sign or None, E4M3 uint8 [M, 32*ld] or None, scale [M])."""
+    lib = _L()
+    assert X.is_cuda and X.dtype == torch.float16 and X.dim() == 2 and X.stride(1) == 1
+    M, K = X.shape
+    ld = ld_words_for(K)
+    if out is None:
+        mask = torch.empty((M, ld), dtype=torch.int32, device=X.device) if planes else None
+        sign = torch.empty((M, ld), dtype=torch.int32, device=X.device) if planes else None
+        a8 = torch.empty((M, 32 * ld), dtype=torch.uint8, device=X.device) if e4m3 else None
+        scale = torch.empty((M,), dtype=torch.float32, device=X.device)
+    else:
+        mask, sign, a8, scale = out
+    _check("bwta_quantize_pack_acts_ex", lib.bwta_quantize_pack_acts_ex(
+        _ptr(X), M, K, _row_stride(X), mode, thresh_ratio, _ptr(mask), _ptr(sign), ld, _ptr(a8),
+        a8.shape[1] if a8 is not None else 0, _ptr(scale), _ptr(status), _stream()))
+    return mask, sign, a8, scale
+
+
+def bwta_gemm_tc(a_e4m3, a_scale, wbits, wscale, K: int, group: int = 0, want_y: bool = True,
+                 want_dots: bool = False, status=None, out=None):
+    """Tensor-core GEMM on E4M3 activations. Returns (Y fp32 [M, N] or None, dots or None)."""
+    lib = _L()
+    M, ld8 = a_e4m3.shape
+    N, ldw = wbits.shape
+    if out is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=a_e4m3.device) if want_y else None
+        D = torch.empty((M, N), dtype=torch.int32, device=a_e4m3.device) if want_dots else None
+    else:
+        Y, D = out
+    _check("bwta_gemm_tc", lib.bwta_gemm_tc(
+        _ptr(a_e4m3), ld8, _ptr(a_scale), M, _ptr(wbits), _ptr(wscale), N, ldw, K, group, _ptr(Y),
+        _row_stride(Y) if Y is not None else N, _ptr(D), _row_stride(D) if D is not None else N,
+        _ptr(status), _stream()))
+    return Y, D
 
 
 def bwta_gemm(a_mask, a_sign, a_scale, wbits, wscale, K: int, group: int = 0,

@@ -56,7 +56,52 @@ int bwta_quantize_pack_acts(const uint16_t *X, int64_t M, int64_t K, int64_t ldX
   if (int r = check_plane(mask, M, lda_words, K)) return r;
   if (int r = check_plane(sign, M, lda_words, K)) return r;
   return cuda_status(launch_quantize_pack_acts(X, M, K, ldX, mode, mask, sign, lda_words, scale,
-                                               d_status, (cudaStream_t)stream));
+                                               nullptr, 0, d_status, (cudaStream_t)stream));
+}
+
+int bwta_quantize_pack_acts_ex(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
+                               float thresh_ratio, uint32_t *mask, uint32_t *sign,
+                               int64_t lda_words, uint8_t *a_e4m3, int64_t ld_e4m3, float *scale,
+                               int32_t *d_status, bwta_stream_t stream) {
+  if (M < 0 || K <= 0 || ldX < K) return BWTA_ERR_INVALID_ARG;
+  if (mode != BWTA_TERNARY && mode != BWTA_BINARY) return BWTA_ERR_INVALID_ARG;
+  if (thresh_ratio != 0.5f || K > BWTA_MAX_K) return BWTA_ERR_UNSUPPORTED;
+  if (M > 0 && (!X || !scale)) return BWTA_ERR_INVALID_ARG;
+  if ((mask == nullptr) != (sign == nullptr)) return BWTA_ERR_INVALID_ARG;
+  if (!mask && !a_e4m3) return BWTA_ERR_INVALID_ARG;
+  if (lda_words < words_for(K)) return BWTA_ERR_INVALID_ARG;
+  if (lda_words % 4 != 0) return BWTA_ERR_ALIGNMENT;
+  if (mask) {
+    if (int r = check_plane(mask, M, lda_words, K)) return r;
+    if (int r = check_plane(sign, M, lda_words, K)) return r;
+  }
+  if (a_e4m3) {
+    if (ld_e4m3 < lda_words * 32) return BWTA_ERR_INVALID_ARG;
+    if (ld_e4m3 % 16 != 0 || !aligned16(a_e4m3)) return BWTA_ERR_ALIGNMENT;
+  }
+  return cuda_status(launch_quantize_pack_acts(X, M, K, ldX, mode, mask, sign, lda_words, scale,
+                                               a_e4m3, ld_e4m3, d_status, (cudaStream_t)stream));
+}
+
+int bwta_gemm_tc(const uint8_t *a_e4m3, int64_t ld_e4m3, const float *a_scale, int64_t M,
+                 const uint32_t *wbits, const float *wscale, int64_t N, int64_t ldw_words, int64_t K,
+                 int64_t group, float *Y, int64_t ldY, int32_t *dots, int64_t ldD,
+                 int32_t *d_status, bwta_stream_t stream) {
+  if (M < 0 || N < 0 || K <= 0) return BWTA_ERR_INVALID_ARG;
+  if (K > BWTA_MAX_K) return BWTA_ERR_UNSUPPORTED;
+  if (int r = check_group(group)) return r;
+  if (!Y && !dots) return BWTA_ERR_INVALID_ARG;
+  if (Y && ldY < N) return BWTA_ERR_INVALID_ARG;
+  if (dots && ldD < N) return BWTA_ERR_INVALID_ARG;
+  if (M > 0 && Y && !a_scale) return BWTA_ERR_INVALID_ARG;
+  if (N > 0 && !wscale) return BWTA_ERR_INVALID_ARG;
+  if (M > 0 && !a_e4m3) return BWTA_ERR_INVALID_ARG;
+  if (ld_e4m3 < ((K + 127) / 128) * 128) return BWTA_ERR_INVALID_ARG;
+  if (ld_e4m3 % 16 != 0 || !aligned16(a_e4m3)) return BWTA_ERR_ALIGNMENT;
+  if (int r = check_plane(wbits, N, ldw_words, K)) return r;
+  if (M == 0 || N == 0) return BWTA_OK;
+  return cuda_status(launch_gemm_tc(a_e4m3, ld_e4m3, a_scale, M, wbits, wscale, N, ldw_words, K,
+                                    group, Y, ldY, dots, ldD, d_status, (cudaStream_t)stream));
 }
 
 int bwta_gemm(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_scale, int64_t M,

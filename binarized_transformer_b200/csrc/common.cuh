@@ -118,7 +118,12 @@ cudaError_t launch_pack_weights(const float *W, int64_t N, int64_t K, int64_t ld
                                 cudaStream_t s);
 cudaError_t launch_quantize_pack_acts(const uint16_t *X, int64_t M, int64_t K, int64_t ldX,
                                       int mode, uint32_t *mask, uint32_t *sign, int64_t lda,
-                                      float *scale, int32_t *d_status, cudaStream_t s);
+                                      float *scale, uint8_t *a8, int64_t ld8, int32_t *d_status,
+                                      cudaStream_t s);
+cudaError_t launch_gemm_tc(const uint8_t *a8, int64_t ld8, const float *ascale, int64_t M,
+                           const uint32_t *wb, const float *wscale, int64_t N, int64_t ldw,
+                           int64_t K, int64_t group, float *Y, int64_t ldY, int32_t *dots,
+                           int64_t ldD, int32_t *d_status, cudaStream_t s);
 cudaError_t launch_gemm_tiled(const uint32_t *am, const uint32_t *as, const float *ascale,
                               int64_t M, int64_t lda, const uint32_t *wb, const float *wscale,
                               int64_t N, int64_t ldw, int64_t K, int64_t group, float *Y,

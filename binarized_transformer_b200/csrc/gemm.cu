@@ -47,6 +47,21 @@ bool make_plane_map(CUtensorMap *map, const uint32_t *base, int64_t rows, int64_
   return r == CUDA_SUCCESS;
 }
 
+bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, int elem_bytes, const void *base,
+                 int64_t rows, int64_t ld, uint32_t box_w, uint32_t box_h,
+                 CUtensorMapSwizzle swizzle) {
+  PFN_encodeTiled enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * (cuuint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_w, box_h};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ============================================================ tiled GEMM (K2)
 // CTA tile 128 (activation rows) x 128 (weight rows), K staged 32 words
 // (1024 elements) at a time by TMA into a 3-deep ring of 128-byte-swizzled

@@ -104,7 +104,8 @@ template <int T, bool TERNARY, bool VEC>
 __global__ void __launch_bounds__(QA_THREADS)
 k_quantize_pack_acts(const uint16_t *__restrict__ X, int64_t M, int64_t K, int64_t ldX,
                      uint32_t *__restrict__ mask, uint32_t *__restrict__ sign, int64_t lda,
-                     float *__restrict__ scale, int32_t *d_status) {
+                     float *__restrict__ scale, uint8_t *__restrict__ a8, int64_t ld8,
+                     int32_t *d_status) {
   constexpr int TEAMS = QA_THREADS / T;
   constexpr int CPS = T / 16;  // chunks per step
   __shared__ uint64_t red[QA_THREADS / 32];
@@ -139,8 +140,8 @@ k_quantize_pack_acts(const uint16_t *__restrict__ X, int64_t M, int64_t K, int64
 
   // pass 2: threshold, bit planes, kept sums
   const uint32_t hT = TERNARY ? mag_threshold_pattern(S / (uint64_t)(2 * K)) : 0u;
-  uint32_t *mrow = mask + (valid ? row : 0) * lda;
-  uint32_t *srow = sign + (valid ? row : 0) * lda;
+  uint32_t *mrow = mask ? mask + (valid ? row : 0) * lda : nullptr;
+  uint32_t *srow = sign ? sign + (valid ? row : 0) * lda : nullptr;
   uint64_t ks = 0, kn = 0;
 #pragma unroll
   for (int s = 0; s < QA_NREG; ++s) {
@@ -150,7 +151,8 @@ k_quantize_pack_acts(const uint16_t *__restrict__ X, int64_t M, int64_t K, int64
       uint32_t kb, sb;
       keep8<TERNARY>(regs[s], hT, k0, K, kb, sb, ks);
       kn += __popc(kb);
-      store_chunk(kb, sb, mrow, srow, chunk, valid && chunk < C);
+      store_chunk(kb, sb, mrow, srow, chunk, valid && chunk < C && mask);
+      if (a8 && valid && chunk < C) store_e4m3x8(a8 + row * ld8 + k0, kb, sb);
     }
   }
   for (int s = QA_NREG; s < steps; ++s) {
@@ -159,7 +161,8 @@ k_quantize_pack_acts(const uint16_t *__restrict__ X, int64_t M, int64_t K, int64
     uint32_t kb, sb;
     keep8<TERNARY>(load_half8<VEC>(xr, k0, K, valid), hT, k0, K, kb, sb, ks);
     kn += __popc(kb);
-    store_chunk(kb, sb, mrow, srow, chunk, valid && chunk < C);
+    store_chunk(kb, sb, mrow, srow, chunk, valid && chunk < C && mask);
+    if (a8 && valid && chunk < C) store_e4m3x8(a8 + row * ld8 + k0, kb, sb);
   }
 
   // pass 3: row scale
@@ -185,13 +188,13 @@ k_quantize_pack_acts(const uint16_t *__restrict__ X, int64_t M, int64_t K, int64
 template <int T>
 static cudaError_t launch_qa_t(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
                                uint32_t *mask, uint32_t *sign, int64_t lda, float *scale,
-                               int32_t *d_status, cudaStream_t s) {
+                               uint8_t *a8, int64_t ld8, int32_t *d_status, cudaStream_t s) {
   constexpr int TEAMS = QA_THREADS / T;
   const int64_t blocks = ceil_div<int64_t>(M, TEAMS);
   const bool vec = (reinterpret_cast<uintptr_t>(X) & 15u) == 0 && ldX % 8 == 0;
 #define BWTA_QA(TER, V)                                                                          \
   return launch_pdl(k_quantize_pack_acts<T, TER, V>, dim3((unsigned)blocks), dim3(QA_THREADS), 0, s, \
-                    X, M, K, ldX, mask, sign, lda, scale, d_status)
+                    X, M, K, ldX, mask, sign, lda, scale, a8, ld8, d_status)
   if (mode == BWTA_TERNARY) {
     if (vec) BWTA_QA(true, true);
     BWTA_QA(true, false);
@@ -203,14 +206,15 @@ static cudaError_t launch_qa_t(const uint16_t *X, int64_t M, int64_t K, int64_t 
 
 cudaError_t launch_quantize_pack_acts(const uint16_t *X, int64_t M, int64_t K, int64_t ldX,
                                       int mode, uint32_t *mask, uint32_t *sign, int64_t lda,
-                                      float *scale, int32_t *d_status, cudaStream_t s) {
+                                      float *scale, uint8_t *a8, int64_t ld8, int32_t *d_status,
+                                      cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   const int64_t C = lda / 4;  // 128-element chunks per row
-  if (C <= 1) return launch_qa_t<16>(X, M, K, ldX, mode, mask, sign, lda, scale, d_status, s);
-  if (C <= 2) return launch_qa_t<32>(X, M, K, ldX, mode, mask, sign, lda, scale, d_status, s);
-  if (C <= 4) return launch_qa_t<64>(X, M, K, ldX, mode, mask, sign, lda, scale, d_status, s);
-  if (C <= 8) return launch_qa_t<128>(X, M, K, ldX, mode, mask, sign, lda, scale, d_status, s);
-  return launch_qa_t<256>(X, M, K, ldX, mode, mask, sign, lda, scale, d_status, s);
+  if (C <= 1) return launch_qa_t<16>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+  if (C <= 2) return launch_qa_t<32>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+  if (C <= 4) return launch_qa_t<64>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+  if (C <= 8) return launch_qa_t<128>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+  return launch_qa_t<256>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
 }
 
 }  // namespace bwta

@@ -104,6 +104,16 @@ __device__ __forceinline__ void store_chunk(uint32_t kb, uint32_t sb, uint32_t *
 }
 
 
+// E4M3 bytes of 8 ternary values (keep bits kb, sign bits sb; bit i = value i):
+// +1 = 0x38, -1 = 0xB8, 0 = 0x00. spread() moves bit i of a nibble to bit 0 of
+// byte i (the four shifted copies 0, 7, 14, 21 do not overlap).
+__device__ __forceinline__ uint32_t spread_nibble(uint32_t x) { return (x * 0x00204081u) & 0x01010101u; }
+__device__ __forceinline__ void store_e4m3x8(uint8_t *dst, uint32_t kb, uint32_t sb) {
+  const uint32_t lo = spread_nibble(kb & 15u) * 0x38u | spread_nibble(sb & 15u) * 0x80u;
+  const uint32_t hi = spread_nibble(kb >> 4) * 0x38u | spread_nibble(sb >> 4) * 0x80u;
+  *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
+}
+
 // Row scale from the exact kept sum / count (ternary) or the row sum (binary),
 // with the roundings of the definition: int64 -> fp64, fp64 divide, times
 // 2^-24, fp64 -> fp32.

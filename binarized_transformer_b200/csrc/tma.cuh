@@ -26,6 +26,12 @@ PFN_encodeTiled get_encode_tiled();
 bool make_plane_map(CUtensorMap *map, const uint32_t *base, int64_t rows, int64_t ld,
                     uint32_t box_w, uint32_t box_h);
 
+// A 2-D map over a row-major matrix [rows][ld] of `elem_bytes`-byte elements
+// (dtype UINT8 or UINT32), box = box_w x box_h elements, the given swizzle.
+bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, int elem_bytes, const void *base,
+                 int64_t rows, int64_t ld, uint32_t box_w, uint32_t box_h,
+                 CUtensorMapSwizzle swizzle);
+
 // ---------------------------------------------------------------- device
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);

@@ -96,6 +96,39 @@ int bwta_quantize_pack_acts(const uint16_t *X, int64_t M, int64_t K, int64_t ldX
                             int64_t lda_words, float *scale, int32_t *d_status,
                             bwta_stream_t stream);
 
+/* bwta_quantize_pack_acts that can also (or only) write the ternary values as
+ * 8-bit floats for the tensor-core GEMM: one E4M3 byte per element, +1 = 0x38,
+ * -1 = 0xB8, 0 = 0x00 (same keep/sign decisions, same scale).
+ *  mask, sign     both NULL or both valid (uint32 [M][lda_words])
+ *  a_e4m3         uint8 [M][ld_e4m3] out, may be NULL (not together with mask);
+ *                 bytes 0 .. 32*lda_words-1 of every row are written, those past
+ *                 K as 0; ld_e4m3 >= 32*lda_words, ld_e4m3 % 16 == 0
+ *  lda_words      row stride of the planes; also fixes how many E4M3 bytes
+ *                 per row are written
+ *  Errors: as bwta_quantize_pack_acts. */
+int bwta_quantize_pack_acts_ex(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
+                               float thresh_ratio, uint32_t *mask, uint32_t *sign,
+                               int64_t lda_words, uint8_t *a_e4m3, int64_t ld_e4m3, float *scale,
+                               int32_t *d_status, bwta_stream_t stream);
+
+/* The same product as bwta_gemm on the tensor cores (tcgen05.mma, 8-bit
+ * floating-point operands, fp32 accumulation). Every +-1 x {-1,0,+1} product
+ * and partial sum is an integer below 2^24 and therefore exact, so the dots
+ * are the same integers and Y follows the same fp32 order (group by group,
+ * then the activation scale): the outputs equal bwta_gemm's tiled path bit
+ * for bit. The weights stay bit-packed in memory and are expanded to E4M3
+ * inside the kernel.
+ *  a_e4m3, ld_e4m3  activations from bwta_quantize_pack_acts_ex
+ *                   (ld_e4m3 >= 128 * ceil(K/128), % 16 == 0, 16-byte aligned)
+ *  a_scale          fp32 [M] (may be NULL when Y is NULL)
+ *  other arguments  as bwta_gemm (group 0 or a multiple of 128)
+ *  d_status         BWTA_STATUS_TIMEOUT if a bounded barrier wait gave up
+ *  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA. */
+int bwta_gemm_tc(const uint8_t *a_e4m3, int64_t ld_e4m3, const float *a_scale, int64_t M,
+                 const uint32_t *wbits, const float *wscale, int64_t N, int64_t ldw_words, int64_t K,
+                 int64_t group, float *Y, int64_t ldY, int32_t *dots, int64_t ldD,
+                 int32_t *d_status, bwta_stream_t stream);
+
 /* Bit-packed GEMM: Y = (s_a * A_ternary) x (alpha * B_binary)^T
  * (BWTA abstract: the bit-packed binary/ternary MatMul for linear layers).
  * Per output (m, n) and weight group g over the words of that group:
