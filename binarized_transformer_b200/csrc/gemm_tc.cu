@@ -10,21 +10,32 @@
 // the same order (acc = fma((float)d_g, alpha_g, acc) over the weight groups,
 // times the activation scale), so its fp32 outputs match bit for bit.
 //
-// Layout (one CTA = 128 weight rows x 128 tokens, 1 CTA per SM):
-//  * the weight rows are the MMA's M dimension and live in TMEM as operand A:
-//    four "expand" warps read each row's sign bits (TMA-loaded, 16 bytes per
-//    row per 128-column block), turn them into E4M3 +-1 bytes through a
-//    16-entry table and store them with tcgen05.st (one lane per row);
-//  * the activations are operand B: E4M3 bytes written by the activation
-//    packer, TMA-loaded 128 tokens x 128 bytes with the 128-byte swizzle;
-//  * the accumulator of one weight group is D (fp32, 128 lanes x 128
-//    columns, three buffers); eight epilogue warps (two per TMEM lane
-//    quarter, 64 token columns each) load a finished group with two
-//    tcgen05.ld, release the buffer, and fold it into running fp32 sums held in
-//    registers; the group scales are prefetched one group ahead;
-//  * one warp issues the TMA loads and the MMAs (one elected thread).
+// Persistent kernel, one CTA per SM, tiles of 128 weight rows x 128 tokens
+// handed out round-robin; every ring below runs on across tile boundaries, so
+// the loads and MMAs of the next tile overlap the last groups and the stores
+// of the current one. Warp roles:
+//  * warp 12 (one thread) issues the TMA loads of each 128-column k-block:
+//    128 tokens x 128 E4M3 bytes of activations (128-byte swizzle) and the
+//    weight rows' sign bits (16 bytes per row), into an 8-stage ring;
+//  * warps 0-3 expand the sign bits into E4M3 +-1 in TMEM (operand A, one TMEM
+//    lane per weight row, 4 buffers). Weight k + 8j of a 32-column block goes
+//    to byte j of word k, the order in which the activation packer writes its
+//    E4M3 bytes, so a word costs one shift and one LOP3;
+//  * warp 13 (one thread) issues 4 MMAs (M=128, N=128, K=32) per k-block into
+//    one of three fp32 accumulators in TMEM (one per weight group in flight);
+//  * warps 4-11 fold each finished group into running fp32 sums in registers
+//    (two warps per TMEM lane quarter, 64 tokens each) and write Y at the end
+//    of a tile.
+// MMA issue blocks until the tensor pipe takes the instruction and the pipe
+// queues little, so the issuing thread does as little as possible between
+// MMAs: one commit per k-block, into a ring of "k-block done" barriers that
+// frees the smem stage, the A buffer and (for groups of at most two
+// k-blocks) signals the finished accumulator all at once; and the barriers of
+// the next k-block are tested, without blocking, before the MMAs of the current
+// one are issued, so that test's latency hides behind them.
 // Every mbarrier wait is bounded (bwta::mbar_wait); on a timeout the CTA
-// records BWTA_STATUS_TIMEOUT and drains.
+// records BWTA_STATUS_TIMEOUT, lets its loads in flight land and its MMAs
+// finish, frees TMEM and returns.
 #include <algorithm>
 
 #include "common.cuh"
@@ -33,42 +44,42 @@
 
 namespace bwta {
 
-constexpr int TC_BM = 128;        // weight rows per CTA (TMEM lanes, MMA M)
-constexpr int TC_BN = 128;        // tokens per CTA (MMA N)
-constexpr int TC_KB = 128;        // K elements per block = one 128-byte swizzle row
-constexpr int TC_STAGES = 7;  // > half the SM's shared memory: one CTA (one TMEM owner) per SM
-constexpr int TC_THREADS = 416;   // warps 0-3 expand, 4-11 epilogue, 12 TMA + MMA
-constexpr int TC_ISSUER = 12;
-constexpr int TC_DBUF = 3;        // accumulator buffers: the MMAs may run two groups ahead
-constexpr int TC_ABUF = 4;        // expanded-weight buffers: expansion may run three blocks ahead
-constexpr int TC_X_BYTES = TC_BN * TC_KB;     // 16 KB of E4M3 activations per stage
-constexpr int TC_W_BYTES = TC_BM * 16;        // 2 KB of weight sign bits per stage
+constexpr int TC_BM = 128;      // weight rows per tile (TMEM lanes, MMA M)
+constexpr int TC_BN = 128;      // tokens per tile (MMA N)
+constexpr int TC_KB = 128;      // K elements per k-block = one 128-byte swizzle row
+constexpr int TC_STAGES = 8;    // smem ring of (activations, weight bits) k-blocks
+constexpr int TC_ABUF = 4;      // expanded-weight buffers in TMEM
+constexpr int TC_DBUF = 3;      // fp32 accumulators in TMEM
+constexpr int TC_PRODUCER = 12, TC_ISSUER = 13;
+constexpr int TC_THREADS = 14 * 32;
+constexpr int TC_X_BYTES = TC_BN * TC_KB;  // 16 KB of E4M3 activations per stage
+constexpr int TC_W_BYTES = TC_BM * 16;     // 2 KB of weight sign bits per stage
 constexpr int TC_STAGE_BYTES = TC_X_BYTES + TC_W_BYTES;
-// TMEM columns: D0 0..127, D1 128..255, D2 256..383, A0..A3 384..511 (32 each)
-constexpr uint32_t TC_TMEM_COLS = 512, TC_COL_A = 384;
+// TMEM columns: D0..D2 at 0, 128, 256; A0..A3 at 384 + 32 b.
+constexpr uint32_t TC_TMEM_COLS = 512, TC_COL_A = TC_DBUF * TC_BN;
 constexpr size_t TC_SMEM = 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES + 1024;
+static_assert(TC_COL_A + TC_ABUF * 32 <= TC_TMEM_COLS, "TMEM budget");
+static_assert(TC_STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned");
+// done[g % TC_STAGES] completes once per k-block g. A thread waiting there for
+// k-block g must not find the phase of k-block g + TC_STAGES completed as well;
+// that cannot happen when k-block g + TC_STAGES needs something the waiter
+// provides after its wait: the producer's load (always), the expand warps'
+// A buffer (TC_STAGES >= TC_ABUF) and the epilogue's accumulator release
+// (groups of seg_len k-blocks with TC_STAGES >= TC_DBUF * seg_len; longer
+// groups get their own commit on d_full).
+static_assert(TC_STAGES >= TC_ABUF && TC_STAGES >= 2 * TC_DBUF, "ring sizes");
+constexpr int TC_SHORT_GROUP = TC_STAGES / TC_DBUF;  // longest group signalled through done[]
 
 struct TcBarriers {
-  uint64_t full[TC_STAGES];   // TMA landed (tx bytes)
-  uint64_t empty[TC_STAGES];  // MMA done with the stage (commit) + 4 expand warps done
+  uint64_t full[TC_STAGES];   // TMA landed (transaction bytes)
+  uint64_t done[TC_STAGES];   // MMAs of k-block g (and all before) complete (commit)
   uint64_t a_full[TC_ABUF];   // expanded weights in TMEM (4 expand warps)
-  uint64_t a_empty[TC_ABUF];  // MMA done with the A buffer (commit)
-  uint64_t d_full[TC_DBUF];   // group accumulated (commit)
-  uint64_t d_empty[TC_DBUF];  // epilogue has read the D buffer (8 epilogue warps)
+  uint64_t d_full[TC_DBUF];   // long group accumulated (commit)
+  uint64_t d_empty[TC_DBUF];  // epilogue has read the accumulator (8 epilogue warps)
+  uint64_t drain;             // all MMAs of the CTA complete (teardown)
   uint32_t tmem_base;
   int32_t timeout;
 };
-
-__device__ __forceinline__ uint64_t *bar_of(TcBarriers *b, int which, int i) {
-  switch (which) {
-    case 0: return &b->full[i];
-    case 1: return &b->empty[i];
-    case 2: return &b->a_full[i];
-    case 3: return &b->a_empty[i];
-    case 4: return &b->d_full[i];
-    default: return &b->d_empty[i];
-  }
-}
 
 // Bounded wait that also records a timeout for the whole CTA.
 __device__ __forceinline__ bool tc_wait(TcBarriers *b, uint64_t *bar, uint32_t parity) {
@@ -78,15 +89,39 @@ __device__ __forceinline__ bool tc_wait(TcBarriers *b, uint64_t *bar, uint32_t p
   return false;
 }
 
-// E4M3 encodings: +1.0 = 0x38, -1.0 = 0xB8, 0 = 0x00. Table entry n holds the
-// four bytes of four weights whose sign bits are the nibble n (bit i = weight i,
-// 1 = negative).
-__device__ __forceinline__ uint32_t e4m3_pm1_word(uint32_t nib) {
-  uint32_t w = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) w |= (((nib >> i) & 1u) ? 0xB8u : 0x38u) << (8 * i);
-  return w;
+// Four E4M3 weights +-1 from the sign-bit word w: byte j is weight 8j + k
+// (sign bit 1 = -1 = 0xB8, 0 = +1 = 0x38).
+template <int k>
+__device__ __forceinline__ uint32_t e4m3_pm1_tc(uint32_t w) {
+  return ((w << (7 - k)) & 0x80808080u) | 0x38383838u;
 }
+
+// Position of the MMA issuer in the (tile, k-block) sequence of its CTA.
+struct TcCursor {
+  int64_t tile;
+  int kb, pos;       // k-block within the tile, within the current group
+  uint32_t g, sg;    // k-blocks and groups before this one (all tiles)
+  bool first, last;  // first / last k-block of its group
+
+  __device__ void set_flags(int KB, int seg_len) {
+    first = pos == 0;
+    last = pos == seg_len - 1 || kb == KB - 1;
+  }
+  __device__ void advance(int KB, int seg_len, int64_t stride) {
+    ++g;
+    if (last) {
+      ++sg;
+      pos = 0;
+    } else {
+      ++pos;
+    }
+    if (++kb == KB) {
+      kb = 0;
+      tile += stride;
+    }
+    set_flags(KB, seg_len);
+  }
+};
 
 template <bool GROUPED, bool WANT_Y, bool WANT_DOTS>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -95,16 +130,15 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
           int KB, int seg_len, int64_t G, float *__restrict__ Y, int64_t ldY,
           int32_t *__restrict__ dots, int64_t ldD, int32_t *d_status) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
+  uint8_t *stages = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *stages = smem;
-  TcBarriers *bars = reinterpret_cast<TcBarriers *>(smem + TC_STAGES * TC_STAGE_BYTES);
-  uint32_t *lut = reinterpret_cast<uint32_t *>(bars + 1);
-  float *sA = reinterpret_cast<float *>(lut + 16);
+  TcBarriers *bars = reinterpret_cast<TcBarriers *>(stages + TC_STAGES * TC_STAGE_BYTES);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t n0 = (int64_t)blockIdx.x * TC_BM, m0 = (int64_t)blockIdx.y * TC_BN;
+  const int64_t NB = ceil_div<int64_t>(N, TC_BM);
+  const int64_t ntiles = NB * ceil_div<int64_t>(M, TC_BN);
   const int nseg = (KB + seg_len - 1) / seg_len;
+  const bool short_group = seg_len <= TC_SHORT_GROUP;  // accumulator signalled through done[]
 
   pdl_trigger();
   if (threadIdx.x == 0) {
@@ -112,126 +146,189 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
     prefetch_tensormap(&map_w);
     for (int s = 0; s < TC_STAGES; ++s) {
       mbar_init(&bars->full[s], 1);
-      mbar_init(&bars->empty[s], 1 + 4);
+      mbar_init(&bars->done[s], 1);
     }
-    for (int i = 0; i < TC_ABUF; ++i) {
-      mbar_init(&bars->a_full[i], 4);
-      mbar_init(&bars->a_empty[i], 1);
-    }
+    for (int i = 0; i < TC_ABUF; ++i) mbar_init(&bars->a_full[i], 4);
     for (int i = 0; i < TC_DBUF; ++i) {
       mbar_init(&bars->d_full[i], 1);
       mbar_init(&bars->d_empty[i], 8);
     }
+    mbar_init(&bars->drain, 1);
     bars->timeout = 0;
     mbar_fence_init();
   }
-  if (threadIdx.x < 16) lut[threadIdx.x] = e4m3_pm1_word(threadIdx.x);
   if (warp == TC_ISSUER) {
     tmem_alloc(&bars->tmem_base, TC_TMEM_COLS);
     tmem_relinquish();
   }
   pdl_wait();
-  if (threadIdx.x < TC_BN) sA[threadIdx.x] = (WANT_Y && m0 + threadIdx.x < M) ? __ldg(ascale + m0 + threadIdx.x) : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == TC_ISSUER) {
-    // ------------------------------------------------ TMA + MMA issuer
+  if (warp == TC_PRODUCER) {
+    // ------------------------------------------------ TMA loads
     if (lane == 0) {
-      auto tma = [&](int kb) -> bool {
-        const int s = kb % TC_STAGES;
-        if (kb >= TC_STAGES && !tc_wait(bars, &bars->empty[s], ((kb / TC_STAGES) - 1) & 1))
-          return false;
-        uint8_t *st = stages + s * TC_STAGE_BYTES;
-        mbar_arrive_expect_tx(&bars->full[s], TC_STAGE_BYTES);
-        tma_load_2d(st, &map_x, kb * TC_KB, (int32_t)m0, &bars->full[s]);
-        tma_load_2d(st + TC_X_BYTES, &map_w, kb * 4, (int32_t)n0, &bars->full[s]);
-        return true;
-      };
-      constexpr int LOOK = TC_STAGES - 2;  // loads run LOOK blocks ahead of the MMAs
+      uint32_t g = 0;  // k-blocks loaded so far (all tiles)
       bool ok = true;
-      for (int kb = 0; kb < LOOK && kb < KB && ok; ++kb) ok = tma(kb);
+      for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int32_t n0 = (int32_t)((tile % NB) * TC_BM), m0 = (int32_t)((tile / NB) * TC_BN);
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % TC_STAGES;
+          // the stage's previous k-block is done (its bits were read before its MMAs)
+          if (g >= TC_STAGES && !tc_wait(bars, &bars->done[s], ((g / TC_STAGES) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          uint8_t *st = stages + s * TC_STAGE_BYTES;
+          mbar_arrive_expect_tx(&bars->full[s], TC_STAGE_BYTES);
+          tma_load_2d(st, &map_x, kb * TC_KB, m0, &bars->full[s]);
+          tma_load_2d(st + TC_X_BYTES, &map_w, kb * 4, n0, &bars->full[s]);
+        }
+      }
+      // Loads still in flight (after a timeout) land before the CTA exits; in
+      // a normal run these phases are complete already.
+      for (uint32_t j = g > TC_STAGES ? g - TC_STAGES : 0; j < g; ++j)
+        mbar_wait(&bars->full[j % TC_STAGES], (j / TC_STAGES) & 1, 100000000ull);
+    }
+    __syncwarp();
+  } else if (warp == TC_ISSUER) {
+    // ------------------------------------------------ MMA issue
+    if (lane == 0) {
       const uint32_t idesc = idesc_e4m3_f32(TC_BM, TC_BN);
-      for (int kb = 0; kb < KB && ok; ++kb) {
-        if (kb + LOOK < KB && !tma(kb + LOOK)) break;
-        const int seg = kb / seg_len, d = seg % TC_DBUF, s = kb % TC_STAGES, b = kb % TC_ABUF;
-        const bool first = (kb % seg_len) == 0;
-        const bool last = (kb % seg_len) == seg_len - 1 || kb == KB - 1;
-        if (first && seg >= TC_DBUF &&
-            !tc_wait(bars, &bars->d_empty[d], ((seg / TC_DBUF) - 1) & 1))
-          break;
-        if (!tc_wait(bars, &bars->full[s], (kb / TC_STAGES) & 1)) break;
-        if (!tc_wait(bars, &bars->a_full[b], (kb / TC_ABUF) & 1)) break;
+      // Non-blocking test of everything k-block c needs.
+      auto ready = [&](const TcCursor &c) -> bool {
+        bool r = mbar_test(&bars->full[c.g % TC_STAGES], (c.g / TC_STAGES) & 1) &
+                 mbar_test(&bars->a_full[c.g % TC_ABUF], (c.g / TC_ABUF) & 1);
+        if (c.first && c.sg >= TC_DBUF)
+          r &= mbar_test(&bars->d_empty[c.sg % TC_DBUF], ((c.sg / TC_DBUF) - 1) & 1);
+        return r;
+      };
+      // Blocking (bounded) version of the same.
+      auto wait_all = [&](const TcCursor &c) -> bool {
+        if (c.first && c.sg >= TC_DBUF &&
+            !tc_wait(bars, &bars->d_empty[c.sg % TC_DBUF], ((c.sg / TC_DBUF) - 1) & 1))
+          return false;
+        return tc_wait(bars, &bars->full[c.g % TC_STAGES], (c.g / TC_STAGES) & 1) &&
+               tc_wait(bars, &bars->a_full[c.g % TC_ABUF], (c.g / TC_ABUF) & 1);
+      };
+      TcCursor cur{(int64_t)blockIdx.x, 0, 0, 0u, 0u, true, true};
+      cur.set_flags(KB, seg_len);
+      bool rdy = cur.tile < ntiles && ready(cur);
+      while (cur.tile < ntiles) {
+        if (!rdy && !wait_all(cur)) break;
         tc_fence_after();
-        const uint32_t xs = smem_addr(stages + s * TC_STAGE_BYTES);
+        TcCursor nxt = cur;
+        nxt.advance(KB, seg_len, gridDim.x);
+        rdy = nxt.tile < ntiles && ready(nxt);  // result needed only after the MMAs below
+        const int d = cur.sg % TC_DBUF, b = cur.g % TC_ABUF;
+        const uint32_t xs = smem_addr(stages + (cur.g % TC_STAGES) * TC_STAGE_BYTES);
 #pragma unroll
         for (int k4 = 0; k4 < TC_KB / 32; ++k4)
-          mma_f8f6f4_ts(tmem + d * 128, tmem + TC_COL_A + b * 32 + k4 * 8,
-                        smem_desc_k_sw128(xs + k4 * 32), idesc, (first && k4 == 0) ? 0u : 1u);
-        tc_commit(&bars->empty[s]);
-        tc_commit(&bars->a_empty[b]);
-        if (last) tc_commit(&bars->d_full[d]);
+          mma_f8f6f4_ts(tmem + d * TC_BN, tmem + TC_COL_A + b * 32 + k4 * 8,
+                        smem_desc_k_sw128(xs + k4 * 32), idesc, (cur.first && k4 == 0) ? 0u : 1u);
+        tc_commit(&bars->done[cur.g % TC_STAGES]);
+        if (cur.last && !short_group) tc_commit(&bars->d_full[d]);
+        cur = nxt;
       }
+      // Every MMA issued has completed before TMEM is released.
+      tc_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, 100000000ull);
     }
     __syncwarp();
   } else if (warp < 4) {
     // ------------------------------------------------ weight bits -> E4M3 in TMEM
     const int r = warp * 32 + lane;
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % TC_STAGES, b = kb % TC_ABUF;
-      bool ok = tc_wait(bars, &bars->full[s], (kb / TC_STAGES) & 1);
-      if (ok && kb >= TC_ABUF) ok = tc_wait(bars, &bars->a_empty[b], ((kb / TC_ABUF) - 1) & 1);
-      if (!__all_sync(FULL, ok)) break;
-      const uint4 bits = *reinterpret_cast<const uint4 *>(stages + s * TC_STAGE_BYTES + TC_X_BYTES + r * 16);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->empty[s]);
-      const uint32_t wd[4] = {bits.x, bits.y, bits.z, bits.w};
-      uint32_t v[32];
+    uint32_t g = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb, ++g) {
+        const int s = g % TC_STAGES, b = g % TC_ABUF;
+        bool fine = tc_wait(bars, &bars->full[s], (g / TC_STAGES) & 1);
+        if (fine && g >= TC_ABUF)  // the A buffer's previous k-block is done
+          fine = tc_wait(bars, &bars->done[(g - TC_ABUF) % TC_STAGES],
+                         ((g - TC_ABUF) / TC_STAGES) & 1);
+        if (!__all_sync(FULL, fine)) {
+          ok = false;
+          break;
+        }
+        const uint4 bits =
+            *reinterpret_cast<const uint4 *>(stages + s * TC_STAGE_BYTES + TC_X_BYTES + r * 16);
+        uint32_t v[32];
+        const uint32_t wd[4] = {bits.x, bits.y, bits.z, bits.w};
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = lut[(wd[j >> 3] >> (4 * (j & 7))) & 15u];
-      tmem_st32(tmem_addr(tmem, warp * 32, TC_COL_A + b * 32), v);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->a_full[b]);
+        for (int q = 0; q < 4; ++q) {
+          v[8 * q + 0] = e4m3_pm1_tc<0>(wd[q]);
+          v[8 * q + 1] = e4m3_pm1_tc<1>(wd[q]);
+          v[8 * q + 2] = e4m3_pm1_tc<2>(wd[q]);
+          v[8 * q + 3] = e4m3_pm1_tc<3>(wd[q]);
+          v[8 * q + 4] = e4m3_pm1_tc<4>(wd[q]);
+          v[8 * q + 5] = e4m3_pm1_tc<5>(wd[q]);
+          v[8 * q + 6] = e4m3_pm1_tc<6>(wd[q]);
+          v[8 * q + 7] = e4m3_pm1_tc<7>(wd[q]);
+        }
+        tmem_st32(tmem_addr(tmem, warp * 32, TC_COL_A + b * 32), v);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->a_full[b]);
+      }
     }
   } else {
     // ------------------------------------------------ epilogue: fold groups, write Y
     const int h = (warp - 4) / 4, q = warp % 4, r = q * 32 + lane;
-    const int64_t n = n0 + r;
-    float y[64];
-    uint32_t dv0[32], dv1[32];
-    float alpha = (n < N) ? __ldg(wscale + (GROUPED ? n * G : n)) : 0.0f;
-    for (int seg = 0; seg < nseg; ++seg) {
-      const int d = seg % TC_DBUF;
-      const float alpha_next =
-          (GROUPED && seg + 1 < nseg && n < N) ? __ldg(wscale + n * G + seg + 1) : 0.0f;
-      const bool ok = tc_wait(bars, &bars->d_full[d], (seg / TC_DBUF) & 1);
-      if (!__all_sync(FULL, ok)) break;
-      tc_fence_after();
-      tmem_ld32(tmem_addr(tmem, q * 32, d * 128 + h * 64), dv0);
-      tmem_ld32(tmem_addr(tmem, q * 32, d * 128 + h * 64 + 32), dv1);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->d_empty[d]);
+    uint32_t sg = 0, g0 = 0;  // groups and k-blocks of the tiles before this one
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, g0 += KB) {
+      const int64_t n = (tile % NB) * TC_BM + r, m0 = (tile / NB) * TC_BN + h * 64;
+      float y[64];
+      float alpha = (WANT_Y && n < N) ? __ldg(wscale + (GROUPED ? n * G : n)) : 0.0f;
+      for (int seg = 0; seg < nseg; ++seg, ++sg) {
+        const int d = sg % TC_DBUF;
+        const float alpha_next =
+            (WANT_Y && GROUPED && seg + 1 < nseg && n < N) ? __ldg(wscale + n * G + seg + 1) : 0.0f;
+        bool fine;
+        if (short_group) {  // wait for the group's last k-block
+          const uint32_t ge = g0 + (uint32_t)min((seg + 1) * seg_len, KB) - 1;
+          fine = tc_wait(bars, &bars->done[ge % TC_STAGES], (ge / TC_STAGES) & 1);
+        } else {
+          fine = tc_wait(bars, &bars->d_full[d], (sg / TC_DBUF) & 1);
+        }
+        if (!__all_sync(FULL, fine)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t dv[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        y[i] = fmaf(__uint_as_float(dv0[i]), alpha, seg > 0 ? y[i] : 0.0f);
-        y[32 + i] = fmaf(__uint_as_float(dv1[i]), alpha, seg > 0 ? y[32 + i] : 0.0f);
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(tmem_addr(tmem, q * 32, d * TC_BN + h * 64 + c * 32), dv);
+          tmem_wait_ld();
+          if (c == 1) {  // the accumulator is in registers: hand it back to the MMAs
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->d_empty[d]);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            y[c * 32 + i] = fmaf(__uint_as_float(dv[i]), alpha, seg > 0 ? y[c * 32 + i] : 0.0f);
+          if (WANT_DOTS && seg == nseg - 1 && n < N) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int64_t m = m0 + c * 32 + i;
+              if (m < M) dots[m * ldD + n] = __float2int_rn(__uint_as_float(dv[i]));
+            }
+          }
+        }
+        alpha = alpha_next;
       }
-      alpha = alpha_next;
-    }
-    if (n < N && !bars->timeout) {
+      if (!ok) break;
+      if (WANT_Y && n < N) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int64_t m = m0 + h * 64 + i;
-        if (m < M) {
-          if (WANT_Y) Y[m * ldY + n] = y[i] * sA[h * 64 + i];
-          if (WANT_DOTS)
-            dots[m * ldD + n] = __float2int_rn(__uint_as_float(i < 32 ? dv0[i] : dv1[i - 32]));
+        for (int i = 0; i < 64; ++i) {
+          const int64_t m = m0 + i;
+          if (m < M) Y[m * ldY + n] = y[i] * __ldg(ascale + m);
         }
       }
     }
@@ -255,9 +352,13 @@ static cudaError_t launch_tc_t(const CUtensorMap &mx, const CUtensorMap &mw, con
   static cudaError_t attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM);
   if (attr != cudaSuccess) return attr;
-  dim3 grid((unsigned)ceil_div<int64_t>(N, TC_BM), (unsigned)ceil_div<int64_t>(M, TC_BN));
-  return launch_pdl(kern, grid, dim3(TC_THREADS), TC_SMEM, s, mx, mw, ascale, wscale, M, N, KB,
-                    seg_len, G, Y, ldY, dots, ldD, d_status);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t ntiles = ceil_div<int64_t>(N, TC_BM) * ceil_div<int64_t>(M, TC_BN);
+  const unsigned grid = (unsigned)std::min<int64_t>(ntiles, std::max(sms, 1));
+  return launch_pdl(kern, dim3(grid), dim3(TC_THREADS), TC_SMEM, s, mx, mw, ascale, wscale, M, N,
+                    KB, seg_len, G, Y, ldY, dots, ldD, d_status);
 }
 
 cudaError_t launch_gemm_tc(const uint8_t *a8, int64_t ld8, const float *ascale, int64_t M,

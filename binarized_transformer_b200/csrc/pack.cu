@@ -151,8 +151,8 @@ k_quantize_pack_acts(const uint16_t *__restrict__ X, int64_t M, int64_t K, int64
       uint32_t kb, sb;
       keep8<TERNARY>(regs[s], hT, k0, K, kb, sb, ks);
       kn += __popc(kb);
-      store_chunk(kb, sb, mrow, srow, chunk, valid && chunk < C && mask);
-      if (a8 && valid && chunk < C) store_e4m3x8(a8 + row * ld8 + k0, kb, sb);
+      store_chunk(kb, sb, mrow, srow, chunk, valid && chunk < C && mask,
+                  (a8 && valid && chunk < C) ? a8 + row * ld8 + k0 : nullptr);
     }
   }
   for (int s = QA_NREG; s < steps; ++s) {
@@ -161,8 +161,8 @@ k_quantize_pack_acts(const uint16_t *__restrict__ X, int64_t M, int64_t K, int64
     uint32_t kb, sb;
     keep8<TERNARY>(load_half8<VEC>(xr, k0, K, valid), hT, k0, K, kb, sb, ks);
     kn += __popc(kb);
-    store_chunk(kb, sb, mrow, srow, chunk, valid && chunk < C && mask);
-    if (a8 && valid && chunk < C) store_e4m3x8(a8 + row * ld8 + k0, kb, sb);
+    store_chunk(kb, sb, mrow, srow, chunk, valid && chunk < C && mask,
+                (a8 && valid && chunk < C) ? a8 + row * ld8 + k0 : nullptr);
   }
 
   // pass 3: row scale

@@ -83,16 +83,34 @@ __device__ __forceinline__ void keep8(const uint4 &v, uint32_t hT, int64_t k0, i
   }
 }
 
+// E4M3 word k (k = 0..7) of a 32-element block in the tensor-core order: its
+// byte j (j = 0..3) is element 8j + k of the block, +1 = 0x38, -1 = 0xB8,
+// 0 = 0x00. mw / sw are the block's keep / sign words (bit i = element i).
+// Gathering elements k, k+8, k+16, k+24 into one word is a shift and a mask,
+// which is what lets the GEMM expand weight bits into the same order cheaply.
+__device__ __forceinline__ uint32_t e4m3_tc_word(uint32_t mw, uint32_t sw, int k) {
+  return ((mw >> k) & 0x01010101u) * 0x38u | (((sw >> k) << 7) & 0x80808080u);
+}
+
 // Merge the 8-bit patterns of a 16-lane chunk group into 4 words; lane 0 of
-// the group stores them (one 128-bit store per plane).
+// the group stores them (one 128-bit store per plane). With e4m3_dst set, every
+// lane also writes its 8 bytes of the block's E4M3 words in the tensor-core
+// order (lane j of a 4-lane quad: words 2j and 2j+1, which start at the same
+// byte offset as its 8 elements).
 __device__ __forceinline__ void store_chunk(uint32_t kb, uint32_t sb, uint32_t *mrow,
-                                            uint32_t *srow, int chunk, bool do_store) {
+                                            uint32_t *srow, int chunk, bool do_store,
+                                            uint8_t *e4m3_dst = nullptr) {
   const int l16 = threadIdx.x & 15;
   uint32_t mw = kb << (8 * (l16 & 3)), sw = sb << (8 * (l16 & 3));
   mw |= __shfl_xor_sync(FULL, mw, 1);
   sw |= __shfl_xor_sync(FULL, sw, 1);
   mw |= __shfl_xor_sync(FULL, mw, 2);
   sw |= __shfl_xor_sync(FULL, sw, 2);
+  if (e4m3_dst) {
+    const int j = l16 & 3;
+    *reinterpret_cast<uint2 *>(e4m3_dst) =
+        make_uint2(e4m3_tc_word(mw, sw, 2 * j), e4m3_tc_word(mw, sw, 2 * j + 1));
+  }
   const uint32_t m1 = __shfl_down_sync(FULL, mw, 4), m2 = __shfl_down_sync(FULL, mw, 8),
                  m3 = __shfl_down_sync(FULL, mw, 12);
   const uint32_t s1 = __shfl_down_sync(FULL, sw, 4), s2 = __shfl_down_sync(FULL, sw, 8),
@@ -101,17 +119,6 @@ __device__ __forceinline__ void store_chunk(uint32_t kb, uint32_t sb, uint32_t *
     *reinterpret_cast<uint4 *>(mrow + 4 * chunk) = make_uint4(mw, m1, m2, m3);
     *reinterpret_cast<uint4 *>(srow + 4 * chunk) = make_uint4(sw, s1, s2, s3);
   }
-}
-
-
-// E4M3 bytes of 8 ternary values (keep bits kb, sign bits sb; bit i = value i):
-// +1 = 0x38, -1 = 0xB8, 0 = 0x00. spread() moves bit i of a nibble to bit 0 of
-// byte i (the four shifted copies 0, 7, 14, 21 do not overlap).
-__device__ __forceinline__ uint32_t spread_nibble(uint32_t x) { return (x * 0x00204081u) & 0x01010101u; }
-__device__ __forceinline__ void store_e4m3x8(uint8_t *dst, uint32_t kb, uint32_t sb) {
-  const uint32_t lo = spread_nibble(kb & 15u) * 0x38u | spread_nibble(sb & 15u) * 0x80u;
-  const uint32_t hi = spread_nibble(kb >> 4) * 0x38u | spread_nibble(sb >> 4) * 0x80u;
-  *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
 }
 
 // Row scale from the exact kept sum / count (ternary) or the row sum (binary),

@@ -58,25 +58,42 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-// Wait for phase `parity` of the barrier to complete. Bounded: gives up after
-// about `limit_ns` nanoseconds of waiting and returns false.
+// Wait for phase `parity` of the barrier to complete. Each try_wait carries a
+// suspend-time hint, so a waiting thread sleeps until the phase completes (or
+// about a millisecond passes) instead of polling shared memory, where its
+// polls would compete with the tensor cores and TMA for bandwidth. Bounded:
+// gives up after about `limit_ns` nanoseconds of waiting and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           uint64_t limit_ns = 2000000000ull) {
   const uint32_t a = smem_addr(bar);
   uint32_t done = 0;
   uint64_t t0 = 0;
-  for (uint32_t it = 0;; ++it) {
+  for (;;) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(1000000u)
         : "memory");
     if (done) return true;
-    if (it == 0) t0 = global_ns();
-    else if ((it & 63) == 0 && global_ns() - t0 > limit_ns) return false;
+    const uint64_t t = global_ns();
+    if (t0 == 0) t0 = t;
+    else if (t - t0 > limit_ns) return false;
   }
+}
+
+// Non-blocking test: has phase `parity` of the barrier completed?
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
 }
 
 // 2-D tiled bulk tensor load global -> shared, completion signalled on `bar`.

@@ -98,7 +98,11 @@ int bwta_quantize_pack_acts(const uint16_t *X, int64_t M, int64_t K, int64_t ldX
 
 /* bwta_quantize_pack_acts that can also (or only) write the ternary values as
  * 8-bit floats for the tensor-core GEMM: one E4M3 byte per element, +1 = 0x38,
- * -1 = 0xB8, 0 = 0x00 (same keep/sign decisions, same scale).
+ * -1 = 0xB8, 0 = 0x00 (same keep/sign decisions, same scale). Byte order is
+ * the tensor-core order: within each block of 32 elements (bytes 32b ..
+ * 32b+31 of a row), byte 32b + 4k + j (k = 0..7, j = 0..3) holds element
+ * 32b + 8j + k. bwta_gemm_tc expands the weight bits into the same order; a
+ * dot product does not depend on the order its terms are listed in.
  *  mask, sign     both NULL or both valid (uint32 [M][lda_words])
  *  a_e4m3         uint8 [M][ld_e4m3] out, may be NULL (not together with mask);
  *                 bytes 0 .. 32*lda_words-1 of every row are written, those past

@@ -23,10 +23,21 @@ def _lib():
 
 
 def e4m3_of(a, width):
-    """Expected E4M3 bytes of ternary values a [M, K], zero padded to width."""
-    out = np.zeros((a.shape[0], width), np.uint8)
-    out[:, :a.shape[1]] = np.where(a == 1, 0x38, np.where(a == -1, 0xB8, 0)).astype(np.uint8)
-    return out
+    """Expected E4M3 bytes of ternary values a [M, K], zero padded to width, in
+    the tensor-core order of the header: within each 32-element block, byte
+    4k + j holds element 8j + k."""
+    nat = np.zeros((a.shape[0], width), np.uint8)
+    nat[:, :a.shape[1]] = np.where(a == 1, 0x38, np.where(a == -1, 0xB8, 0)).astype(np.uint8)
+    pos = np.arange(32)
+    elem = 8 * (pos % 4) + pos // 4          # element held by byte position pos
+    blocks = nat.reshape(a.shape[0], width // 32, 32)
+    return blocks[:, :, elem].reshape(a.shape[0], width)
+
+
+def test_e4m3_order_is_a_permutation():
+    elem = 8 * (np.arange(32) % 4) + np.arange(32) // 4
+    assert sorted(elem.tolist()) == list(range(32))
+    assert elem[4 * 3 + 2] == 8 * 2 + 3      # byte 4k + j <- element 8j + k
 
 
 @pytest.mark.parametrize("M,K,kind", [(16, 256, "normal"), (9, 33, "student"), (129, 1000, "student"),
