@@ -88,49 +88,104 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples every 200 ms while running."""
+    """SM clock, power and clock-event (throttle) reasons sampled while the
+    timed region runs: NVML polled from a thread every few milliseconds (the
+    region can be far shorter than nvidia-smi's sampling period), falling back
+    to `nvidia-smi -lms 50`. Read-only queries: no setting is changed."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, cuda_index: int, interval: float = 0.005):
+        self.cuda_index = cuda_index
+        self.interval = interval
+        self.samples = []   # (sm_mhz, power_w, reason_bits)
+        self.max_mhz = None
+        self.source = None
         self.proc = None
+        self._stop = None
+
+    def _nvml_handle(self, nv):
+        n = nv.nvmlDeviceGetCount()
+        if n == 1:
+            return nv.nvmlDeviceGetHandleByIndex(0)
+        uuid = str(getattr(torch.cuda.get_device_properties(self.cuda_index), "uuid", ""))
+        for i in range(n):
+            h = nv.nvmlDeviceGetHandleByIndex(i)
+            u = nv.nvmlDeviceGetUUID(h)
+            u = u.decode() if isinstance(u, bytes) else u
+            if uuid and uuid in u:
+                return h
+        return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._nvml_handle(nv)
+            reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self._stop = threading.Event()
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                             nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                             int(reasons_fn(h))))
+                    except Exception:
+                        pass
+                    self._stop.wait(self.interval)
+
+            self._thread = threading.Thread(target=loop, daemon=True)
+            self._thread.start()
+            self.source = "nvml"
+        except Exception:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.cuda_index}", f"--query-gpu={self.Q}",
+                     "--format=csv,noheader,nounits", "-lms", "50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi"
+            except OSError:
+                self.proc = None
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                out, _ = self.proc.communicate(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                out, _ = self.proc.communicate()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for r in csv.reader(io.StringIO(out or "")):
+                if len(r) < 9:
+                    continue
+                bits = 0
+                for nm, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        bits |= self.BITS[nm]
+                self.samples.append((float(r[1]), float(r[3]), bits))
+                self.max_mhz = float(r[2])
 
     def summary(self):
-        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in rows]
-        reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            for n, v in zip(names, r[5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
-                "reasons": sorted(reasons), "samples": len(rows),
-                "power_w_max": max(float(r[3]) for r in rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"],
+                    "samples": 0, "source": self.source}
+        reasons = sorted(n for n, b in self.BITS.items() if any(s[2] & b for s in self.samples))
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
+                "power_w_max": round(max(s[1] for s in self.samples), 1), "source": self.source}
 
 
 class L2Flusher:

@@ -210,11 +210,28 @@ cudaError_t launch_quantize_pack_acts(const uint16_t *X, int64_t M, int64_t K, i
                                       cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   const int64_t C = lda / 4;  // 128-element chunks per row
-  if (C <= 1) return launch_qa_t<16>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
-  if (C <= 2) return launch_qa_t<32>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
-  if (C <= 4) return launch_qa_t<64>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
-  if (C <= 8) return launch_qa_t<128>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
-  return launch_qa_t<256>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+  // Threads per row. Few rows (decode): wide teams, for latency. Many rows
+  // (prefill): the narrowest team that still holds its row in registers
+  // (at most QA_NREG chunk steps per thread), so that more rows, and more
+  // loads, are in flight per SM.
+  int T;
+  if (M < 1024) {
+    T = C <= 1 ? 16 : C <= 2 ? 32 : C <= 4 ? 64 : C <= 8 ? 128 : 256;
+  } else {
+    T = 256;
+    for (int t = 16; t < 256; t *= 2)
+      if (ceil_div<int64_t>(C, t / 16) <= QA_NREG) {
+        T = t;
+        break;
+      }
+  }
+  switch (T) {
+    case 16: return launch_qa_t<16>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+    case 32: return launch_qa_t<32>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+    case 64: return launch_qa_t<64>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+    case 128: return launch_qa_t<128>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+    default: return launch_qa_t<256>(X, M, K, ldX, mode, mask, sign, lda, scale, a8, ld8, d_status, s);
+  }
 }
 
 }  // namespace bwta

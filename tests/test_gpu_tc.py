@@ -115,3 +115,20 @@ def test_gemm_tc_equals_popcount_path():
     torch.cuda.synchronize()
     assert torch.equal(D1, D2)
     assert torch.equal(Y1.view(torch.int32), Y2.view(torch.int32))
+
+
+@pytest.mark.parametrize("K", [4096, 11008, 1000])
+def test_quantize_pack_acts_ex_many_rows(K):
+    """Many rows take the packer's narrow-team path (at most QA_NREG chunk steps
+    per thread); planes, E4M3 bytes and scales must match the oracle exactly."""
+    M = 1100
+    X = workloads.edge_acts(M, K, "student", tag=K + 7)
+    st = bt.new_status()
+    m, s, a8, sc = bt.bwta_quantize_pack_acts_ex(dev(X), status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    a, s_ref = oracle.quantize_acts(X)
+    np.testing.assert_array_equal(u32(m), oracle.pack_plane(a, m.shape[1], "mask"))
+    np.testing.assert_array_equal(u32(s), oracle.pack_plane(a, s.shape[1], "sign"))
+    np.testing.assert_array_equal(a8.cpu().numpy(), e4m3_of(a, a8.shape[1]))
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
