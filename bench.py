@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import csv
 import io
+import hashlib
 import json
 import os
 import statistics
@@ -85,6 +86,26 @@ def measured_peaks():
             d = json.load(f)
         return d, "measured"
     return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+# DRAM traffic of the tensor-core GEMM per launch, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum of the three prefill launches
+# of `bench.py --steps 2 --warmup 1`, averaged): 11.07, 43.87 and 29.72 MB for
+# K x N = 4096x4096, 4096x11008, 11008x4096 at M = 2048. Valid only for the
+# kernel source it was taken on; reported as null once that file changes.
+TC_TRAFFIC = {"source": "binarized_transformer_b200/csrc/gemm_tc.cu",
+              "sha256": "18a0fd282a85075227c64016d3394eda93a95c9dd1a13419780be6b71707f20a",
+              "bytes_per_launch": 28218027}
+
+
+def tc_traffic():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), TC_TRAFFIC["source"])
+    try:
+        with open(path, "rb") as f:
+            ok = hashlib.sha256(f.read()).hexdigest() == TC_TRAFFIC["sha256"]
+    except OSError:
+        ok = False
+    return TC_TRAFFIC["bytes_per_launch"] if ok else None
 
 
 class ClockSampler:
@@ -457,7 +478,8 @@ def run_ours(args):
         "roofline": ({"bound": "tensor", "kernel": "k_gemm_tc (prefill, 3 shapes)",
                       "achieved": round(achieved, 3), "peak": round(fp8_peak, 1),
                       "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
-                      "peak_source": fp8_src, "traffic": None,
+                      "peak_source": fp8_src, "traffic": tc_traffic(),
+                      "traffic_note": "DRAM bytes per k_gemm_tc launch, mean of the 3 shapes (ncu)",
                       "popc_path_ceiling_tops": round(popc_peak_tops, 1)}
                      if step.prefill_path == "tc" else
                      {"bound": "alu", "kernel": "k_gemm_tiled (prefill, 3 shapes)",
