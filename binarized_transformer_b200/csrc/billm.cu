@@ -163,12 +163,16 @@ cudaError_t launch_billm_pack(const float *W, int64_t ldW, int split, const bill
 //   Ts = sum over the sparse group of (+-x)
 //   T1 = sum over salient columns of b1*x,  T2 = the same with b2
 // and adds alpha_c*(T - Ts - T1) + alpha_sp*Ts + alpha1*T1 + alpha2*T2.
-// The sign flip is an XOR of the fp32 sign bit, so +-x costs one LOP3.
+// The sign flip is an XOR of the fp32 sign bit, so +-x costs one LOP3. T is
+// kept as four partial sums (one per 32-column word) so that the adds of a
+// lane form four independent chains. With one activation row the tile is
+// 4*K bytes and several CTAs share an SM.
 constexpr int BG_THREADS = 256, BG_WARPS = BG_THREADS / 32, BG_MT = 4;
 constexpr size_t BG_SMEM_MAX = 160 * 1024;
+template <int MT> constexpr int bg_ctas_per_sm() { return MT == 1 ? 4 : 1; }
 
 template <int MT>
-__global__ void __launch_bounds__(BG_THREADS, 1)
+__global__ void __launch_bounds__(BG_THREADS, bg_ctas_per_sm<MT>())
 k_billm_gemm(const uint16_t *__restrict__ X, int64_t M, int64_t ldX, const uint32_t *__restrict__ sign,
              const uint32_t *__restrict__ gmap, const uint8_t *__restrict__ res,
              const uint8_t *__restrict__ sal, const float *__restrict__ bscale, int64_t N,
@@ -205,21 +209,30 @@ k_billm_gemm(const uint16_t *__restrict__ X, int64_t M, int64_t ldX, const uint3
         const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gmap + n * ldw) + j);
         const float4 sc = __ldg(reinterpret_cast<const float4 *>(bscale) + n * nb + j);
         const uint32_t rb = res[n * nb + j];
-        float T[MT], Ts[MT], T1[MT], T2[MT];
+        float T[MT], Ts[MT], T1[MT], T2[MT], Tq[4][MT];
 #pragma unroll
-        for (int m = 0; m < MT; ++m) T[m] = Ts[m] = T1[m] = T2[m] = 0.0f;
+        for (int m = 0; m < MT; ++m) {
+          T[m] = Ts[m] = T1[m] = T2[m] = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) Tq[q][m] = 0.0f;
+        }
         const uint32_t swa[4] = {sw.x, sw.y, sw.z, sw.w}, gwa[4] = {gw.x, gw.y, gw.z, gw.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t s = swa[q];
 #pragma unroll 8
-          for (int b = 0; b < 32; ++b) {
-            const uint32_t flip = (s << (31 - b)) & 0x80000000u;
+        for (int b = 0; b < 32; ++b) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t flip = (swa[q] << (31 - b)) & 0x80000000u;
             const int c = q * 32 + b;
 #pragma unroll
             for (int m = 0; m < MT; ++m)
-              T[m] += __uint_as_float(__float_as_uint(xs[((size_t)m * 128 + c) * nb + j]) ^ flip);
+              Tq[q][m] += __uint_as_float(__float_as_uint(xs[((size_t)m * 128 + c) * nb + j]) ^ flip);
           }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) T[m] = (Tq[0][m] + Tq[1][m]) + (Tq[2][m] + Tq[3][m]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t s = swa[q];
           uint32_t g = gwa[q];
           while (g) {
             const int b = __ffs(g) - 1;
@@ -276,7 +289,15 @@ static cudaError_t launch_bg_t(const uint16_t *X, int64_t M, int64_t ldX, const 
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BG_SMEM_MAX);
   if (attr != cudaSuccess) return attr;
   const size_t smem = (size_t)MT * W->K * 4 + 8 * (W->K / 128);
-  const int64_t blocks = std::min<int64_t>(ceil_div<int64_t>(W->N, BG_WARPS), 148);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int per_sm = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, BG_THREADS, smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int64_t blocks =
+      std::min<int64_t>(ceil_div<int64_t>(W->N, BG_WARPS), (int64_t)sms * per_sm);
   return launch_pdl(kern, dim3((unsigned)blocks), dim3(BG_THREADS), smem, s, X, M, ldX, W->sign,
                     W->gmap, W->res, W->sal, W->bscale, W->N, W->K, W->ldw_words, (int)W->n_sal, Y,
                     ldY, d_status);
