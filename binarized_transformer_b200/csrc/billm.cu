@@ -306,6 +306,10 @@ static cudaError_t launch_bg_t(const uint16_t *X, int64_t M, int64_t ldX, const 
 cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,
                               float *Y, int64_t ldY, int32_t *d_status, cudaStream_t s) {
   if (M == 0 || W->N == 0) return cudaSuccess;
+  if (M >= 2) {  // tensor cores, when X satisfies the TMA alignment rules
+    const cudaError_t e = launch_billm_gemm_tc(X, M, ldX, W, Y, ldY, d_status, s);
+    if (e != cudaErrorNotSupported) return e;
+  }
   const int mt = billm_gemm_mt(W->K);
   if (mt >= 4 && M >= 4) return launch_bg_t<4>(X, M, ldX, W, Y, ldY, d_status, s);
   if (mt >= 2 && M >= 2) return launch_bg_t<2>(X, M, ldX, W, Y, ldY, d_status, s);

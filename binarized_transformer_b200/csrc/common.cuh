@@ -145,6 +145,8 @@ cudaError_t launch_attn_scores(const uint32_t *qm, const uint32_t *qs, const flo
                                int32_t *Si, float *Sf, cudaStream_t s);
 cudaError_t launch_billm_pack(const float *W, int64_t ldW, int split, const billm_weights *out,
                               int32_t *d_status, cudaStream_t s);
+cudaError_t launch_billm_gemm_tc(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,
+                                 float *Y, int64_t ldY, int32_t *d_status, cudaStream_t s);
 cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,
                               float *Y, int64_t ldY, int32_t *d_status, cudaStream_t s);
 

@@ -381,3 +381,52 @@ def test_billm_full_config(billm_full, M):
     Y = bt.billm_gemm(dev(X), Wq).cpu().numpy()
     yref, mag = billm_rows_ref(X, W, sal, rows)
     assert_close_rel(Y[:, rows], yref, mag, what=f"billm M={M}")
+
+
+@pytest.mark.parametrize("N,K,M", [(200, 384, 300), (129, 128, 70), (64, 1024, 2), (300, 256, 257)])
+def test_billm_tc_shapes(N, K, M):
+    """Tensor-core BiLLM path (M >= 2): ragged token tiles (64 and 256), ragged
+    weight-row tiles, odd block counts."""
+    W = workloads.latent_laplace((N, K), 0.01, 11, N, K)
+    X = workloads.edge_acts(M, K, "student", tag=N + K)
+    Wq = bt.billm_pack_weights(dev(W), n_sal=8, split=True)
+    torch.cuda.synchronize()
+    sal, _ = check_billm_pack(W, Wq, range(N), 8, True)
+    Y = bt.billm_gemm(dev(X), Wq).cpu().numpy()
+    yref, mag = billm_rows_ref(X, W, sal, None, True)
+    assert_close_rel(Y, yref, mag, what=f"billm tc {N}x{K} M={M}")
+
+
+def test_billm_tc_scale_spread():
+    """Rows whose scales differ by many powers of ten, and an all-zero row: the
+    per-row power-of-two exponent keeps every row's hi/lo split in range."""
+    N, K, M = 48, 512, 33
+    W = workloads.latent_laplace((N, K), 0.01, 13, N, K)
+    W = W * (10.0 ** (np.arange(N) % 10 - 6.0))[:, None].astype(np.float32)
+    W[5] = 0.0
+    X = workloads.edge_acts(M, K, "normal", tag=99)
+    Wq = bt.billm_pack_weights(dev(W), n_sal=8, split=True)
+    torch.cuda.synchronize()
+    sal, _ = check_billm_pack(W, Wq, range(N), 8, True)
+    Y = bt.billm_gemm(dev(X), Wq).cpu().numpy()
+    yref, mag = billm_rows_ref(X, W, sal, None, True)
+    assert_close_rel(Y, yref, mag, what="billm tc scale spread")
+    assert np.all(Y[:, 5] == 0.0)
+
+
+def test_billm_unaligned_x_takes_cuda_core_path():
+    """X with a row stride that breaks the TMA rule (ldX % 8 != 0) runs on the
+    CUDA-core kernel; both paths agree with the oracle."""
+    N, K, M = 64, 256, 20
+    W = workloads.latent_laplace((N, K), 0.01, 17, N, K)
+    X = workloads.edge_acts(M, K, "normal", tag=5)
+    Wq = bt.billm_pack_weights(dev(W), n_sal=8, split=True)
+    torch.cuda.synchronize()
+    sal, _ = check_billm_pack(W, Wq, range(N), 8, True)
+    wide = torch.zeros((M, K + 3), dtype=torch.float16, device="cuda")
+    wide[:, :K] = dev(X)
+    Y_core = bt.billm_gemm(wide[:, :K], Wq).cpu().numpy()
+    Y_tc = bt.billm_gemm(dev(X), Wq).cpu().numpy()
+    yref, mag = billm_rows_ref(X, W, sal, None, True)
+    assert_close_rel(Y_core, yref, mag, what="billm cuda-core path")
+    assert_close_rel(Y_tc, yref, mag, what="billm tensor-core path")
