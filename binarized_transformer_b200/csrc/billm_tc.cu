@@ -72,7 +72,7 @@ struct BtSync {
 
 template <int BN>
 constexpr size_t bt_smem() {
-  return 1024 + (size_t)BtShape<BN>::STAGES * BtShape<BN>::STAGE + sizeof(BtSync) + BT_MAX_SAL + 64;
+  return 1024 + (size_t)BtShape<BN>::STAGES * BtShape<BN>::STAGE + sizeof(BtSync) + 64 + BT_MAX_SAL + 64;
 }
 
 __device__ __forceinline__ bool bt_wait(BtSync *b, uint64_t *bar, uint32_t parity) {
@@ -119,7 +119,8 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
   uint8_t *stages = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   BtSync *sy = reinterpret_cast<BtSync *>(stages + S * Sh::STAGE);
-  uint8_t *sal_s = reinterpret_cast<uint8_t *>(sy + 1);
+  uint32_t *sel_lut = reinterpret_cast<uint32_t *>(sy + 1);  // 16 PRMT selectors
+  uint8_t *sal_s = reinterpret_cast<uint8_t *>(sel_lut + 16);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nb = (int)(K / 128), KB = (int)(K / BT_KB);
@@ -148,6 +149,13 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
   }
   pdl_wait();
   for (int i = threadIdx.x; i < nb * n_sal; i += BT_THREADS) sal_s[i] = sal[i];
+  if (threadIdx.x < 16) {
+    // code c = g0 | g1 << 1 | s0 << 2 | s1 << 3 of an element pair -> byte selector
+    // picking pattern g + 2s (+alpha_c, +alpha_sp, -alpha_c, -alpha_sp) for each
+    const uint32_t c = threadIdx.x;
+    const uint32_t i0 = (c & 1u) + ((c >> 1) & 2u), i1 = ((c >> 1) & 1u) + ((c >> 2) & 2u);
+    sel_lut[c] = (2 * i0) | ((2 * i0 + 1) << 4) | ((2 * i1) << 8) | ((2 * i1 + 1) << 12);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -227,7 +235,10 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
       uint32_t rb_next = res[n * nb], rb_next2 = nb > 1 ? res[n * nb + 1] : 0u;
       float4 sc = sc_next;
       uint32_t rb = rb_next;
-      uint32_t pc_h = 0, pc_l = 0, psp_h = 0, psp_l = 0, ppp_h = 0, ppp_l = 0, ppm_h = 0, ppm_l = 0;
+      // byte pools of the four non-salient values (+alpha_c, +alpha_sp, -alpha_c,
+      // -alpha_sp; x 2^E, fp16): hi parts in th0/th1, lo parts in tl0/tl1; and the
+      // salient pair values alpha1 + alpha2, alpha1 - alpha2
+      uint32_t th0 = 0, th1 = 0, tl0 = 0, tl1 = 0, ppp_h = 0, ppp_l = 0, ppm_h = 0, ppm_l = 0;
       for (int kb = 0; kb < KB; ++kb, ++g) {
         const int s = g % S, j = kb >> 1;
         if ((kb & 1) == 0) {  // a new 128-column block: its scales, the next block's in flight
@@ -239,10 +250,15 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
             sc_next2 = __ldg(bs_row + j + 2);
             rb_next2 = res[n * nb + j + 2];
           }
+          uint32_t pc_h, pc_l, psp_h, psp_l;
           bt_split(sc.x * pw, pc_h, pc_l);
           bt_split(sc.y * pw, psp_h, psp_l);
           bt_split((sc.z + sc.w) * pw, ppp_h, ppp_l);
           bt_split((sc.z - sc.w) * pw, ppm_h, ppm_l);
+          th0 = pc_h | (psp_h << 16);
+          th1 = th0 ^ 0x80008000u;
+          tl0 = pc_l | (psp_l << 16);
+          tl1 = tl0 ^ 0x80008000u;
         }
         const uint32_t S_w = s0, G_w = g0;
         s0 = s1;
@@ -255,31 +271,14 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
           s3 = __ldg(srow + 2 * (kb + 4) + h);
           g3 = __ldg(grow + 2 * (kb + 4) + h);
         }
-        // salient columns of this thread's 32 columns, and their residual signs
-        const int cb = (kb & 1) * 64 + h * 32;
-        uint32_t SAL = 0, B2 = 0;
-        for (int i = 0; i < n_sal; ++i) {
-          const int c = (int)sal_s[j * n_sal + i] - cb;
-          if (c >= 0 && c < 32) {
-            SAL |= 1u << c;
-            B2 |= ((rb >> i) & 1u) << c;
-          }
-        }
-        // q = which of the two patterns: group bit, or b1 != b2 at salient columns
-        const uint32_t Q = (SAL & (S_w ^ B2)) | (~SAL & G_w);
+        const int cb = (kb & 1) * 64 + h * 32;  // this thread's 32 columns of block j
         uint32_t hw[16], lw[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          uint32_t ph[2], pl[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const bool sl = (SAL >> (e + u)) & 1u, q = (Q >> (e + u)) & 1u;
-            const uint32_t fl = ((S_w >> (e + u)) & 1u) << 15;
-            ph[u] = (sl ? (q ? ppm_h : ppp_h) : (q ? psp_h : pc_h)) ^ fl;
-            pl[u] = (sl ? (q ? ppm_l : ppp_l) : (q ? psp_l : pc_l)) ^ fl;
-          }
-          hw[e / 2] = ph[0] | (ph[1] << 16);
-          lw[e / 2] = pl[0] | (pl[1] << 16);
+        for (int p = 0; p < 16; ++p) {  // element pair 2p, 2p+1: one byte permute per plane
+          const uint32_t code = ((G_w >> (2 * p)) & 3u) | (((S_w >> (2 * p)) & 3u) << 2);
+          const uint32_t sel = sel_lut[code];
+          hw[p] = __byte_perm(th0, th1, sel);
+          lw[p] = __byte_perm(tl0, tl1, sel);
         }
         // the stage's previous k-block is done with its tiles
         bool fine = true;
@@ -298,6 +297,18 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
               make_uint4(hw[4 * c4], hw[4 * c4 + 1], hw[4 * c4 + 2], hw[4 * c4 + 3]);
           *reinterpret_cast<uint4 *>(alo + off) =
               make_uint4(lw[4 * c4], lw[4 * c4 + 1], lw[4 * c4 + 2], lw[4 * c4 + 3]);
+        }
+        // salient columns: b1 * (alpha1 + alpha2) when b1 == b2, b1 * (alpha1 - alpha2) otherwise
+        for (int i = 0; i < n_sal; ++i) {
+          const int c = (int)sal_s[j * n_sal + i] - cb;
+          if (c >= 0 && c < 32) {
+            const uint32_t b1 = (S_w >> c) & 1u, b2 = (rb >> i) & 1u;
+            const uint32_t vh = (b1 == b2 ? ppp_h : ppm_h) ^ (b1 << 15);
+            const uint32_t vl = (b1 == b2 ? ppp_l : ppm_l) ^ (b1 << 15);
+            const uint32_t off = swz128(r, h * 4 + (c >> 3)) + 2 * (c & 7);
+            *reinterpret_cast<uint16_t *>(ahi + off) = (uint16_t)vh;
+            *reinterpret_cast<uint16_t *>(alo + off) = (uint16_t)vl;
+          }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
