@@ -274,6 +274,147 @@ k_billm_gemm(const uint16_t *__restrict__ X, int64_t M, int64_t ldX, const uint3
   if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
 }
 
+// ------------------------------------------------------------ M = 1 (decode)
+// One activation row: it is staged once per CTA in shared memory as fp32,
+// block-major with a row stride of 132 floats (16-byte aligned, and lanes j
+// reading x[j][c..c+3] hit distinct bank quads), together with the block sums
+// X_j = sum_c x[j][c]. A warp owns a weight row, lane l the blocks l, l+32, ...
+// For a block, sum_c (+-x) = X_j - 2 * sum_{sign bit 1} x: one predicated add
+// per weight, x read four at a time. The sparse group and the salient columns
+// are added as before. The next row's planes and scales are loaded while the
+// current row is summed.
+constexpr int BV_STRIDE = 132;
+
+__global__ void __launch_bounds__(BG_THREADS)
+k_billm_gemv(const uint16_t *__restrict__ X, const uint32_t *__restrict__ sign,
+             const uint32_t *__restrict__ gmap, const uint8_t *__restrict__ res,
+             const uint8_t *__restrict__ sal, const float *__restrict__ bscale, int64_t N,
+             int64_t K, int64_t ldw, int n_sal, float *__restrict__ Y, int32_t *d_status) {
+  extern __shared__ float xs[];  // [nb][BV_STRIDE], then X_j [nb], then salient table
+  pdl_trigger();
+  pdl_wait();
+  const int nb = (int)(K / 128);
+  float *xsum = xs + (size_t)nb * BV_STRIDE;
+  uint8_t *ssal = reinterpret_cast<uint8_t *>(xsum + nb);
+  for (int i = threadIdx.x; i < nb * n_sal; i += BG_THREADS) ssal[i] = sal[i];
+  bool bad = false;
+  for (int64_t k = threadIdx.x; k < K; k += BG_THREADS) {
+    const __half_raw hr = {X[k]};
+    if ((hr.x & 0x7C00u) == 0x7C00u) bad = true;
+    xs[(k >> 7) * BV_STRIDE + (k & 127)] = __half2float(__half(hr));
+  }
+  __syncthreads();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int j = warp; j < nb; j += BG_WARPS) {  // block sums, fp32, fixed order
+    float v = xs[j * BV_STRIDE + lane] + xs[j * BV_STRIDE + lane + 32] +
+              xs[j * BV_STRIDE + lane + 64] + xs[j * BV_STRIDE + lane + 96];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    if (lane == 0) xsum[j] = v;
+  }
+  __syncthreads();
+  if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
+
+  const int64_t stride = (int64_t)gridDim.x * BG_WARPS;
+  int64_t n = (int64_t)blockIdx.x * BG_WARPS + warp;
+  // planes and scales of the first block pair of the first row
+  auto load = [&](int64_t row, int j, uint4 &sw, uint4 &gw, float4 &sc, uint32_t &rb) {
+    if (row < N && j < nb) {
+      sw = __ldg(reinterpret_cast<const uint4 *>(sign + row * ldw) + j);
+      gw = __ldg(reinterpret_cast<const uint4 *>(gmap + row * ldw) + j);
+      sc = __ldg(reinterpret_cast<const float4 *>(bscale) + row * nb + j);
+      rb = res[row * nb + j];
+    } else {
+      sw = gw = make_uint4(0, 0, 0, 0);
+      sc = make_float4(0, 0, 0, 0);
+      rb = 0;
+    }
+  };
+  uint4 sw0, gw0, sw1, gw1;
+  float4 sc0, sc1;
+  uint32_t rb0, rb1;
+  load(n, lane, sw0, gw0, sc0, rb0);
+  load(n, lane + 32, sw1, gw1, sc1, rb1);
+  for (; n < N; n += stride) {
+    // next row in flight
+    uint4 nsw0, ngw0, nsw1, ngw1;
+    float4 nsc0, nsc1;
+    uint32_t nrb0, nrb1;
+    load(n + stride, lane, nsw0, ngw0, nsc0, nrb0);
+    load(n + stride, lane + 32, nsw1, ngw1, nsc1, nrb1);
+    float y = 0.0f;
+    for (int jj = 0; jj < nb; jj += 64) {  // this lane's blocks lane + jj, lane + jj + 32
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int j = lane + jj + half * 32;
+        if (j >= nb) continue;
+        uint4 sw = half ? sw1 : sw0, gw = half ? gw1 : gw0;
+        float4 sc = half ? sc1 : sc0;
+        uint32_t rb = half ? rb1 : rb0;
+        if (jj > 0) load(n, j, sw, gw, sc, rb);  // K > 8192: blocks past the first 64
+        const float *xj = xs + j * BV_STRIDE;
+        const uint32_t swa[4] = {sw.x, sw.y, sw.z, sw.w}, gwa[4] = {gw.x, gw.y, gw.z, gw.w};
+        float neg[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int b4 = 0; b4 < 8; ++b4) {
+            const float4 x4 = *reinterpret_cast<const float4 *>(xj + q * 32 + b4 * 4);
+            const uint32_t s = swa[q] >> (b4 * 4);
+            if (s & 1u) neg[q] += x4.x;
+            if (s & 2u) neg[q] += x4.y;
+            if (s & 4u) neg[q] += x4.z;
+            if (s & 8u) neg[q] += x4.w;
+          }
+        }
+        const float T = xsum[j] - 2.0f * ((neg[0] + neg[1]) + (neg[2] + neg[3]));
+        float Ts = 0.0f, T1 = 0.0f, T2 = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t g = gwa[q];
+          while (g) {
+            const int b = __ffs(g) - 1;
+            g &= g - 1;
+            const uint32_t flip = ((swa[q] >> b) & 1u) << 31;
+            Ts += __uint_as_float(__float_as_uint(xj[q * 32 + b]) ^ flip);
+          }
+        }
+        for (int i = 0; i < n_sal; ++i) {
+          const int c = ssal[j * n_sal + i];
+          const uint32_t xb = __float_as_uint(xj[c]);
+          T1 += __uint_as_float(xb ^ (((swa[c >> 5] >> (c & 31)) & 1u) << 31));
+          T2 += __uint_as_float(xb ^ (((rb >> i) & 1u) << 31));
+        }
+        y += sc.x * (T - Ts - T1) + sc.y * Ts + sc.z * T1 + sc.w * T2;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(FULL, y, o);
+    if (lane == 0) Y[n] = y;
+    sw0 = nsw0; gw0 = ngw0; sc0 = nsc0; rb0 = nrb0;
+    sw1 = nsw1; gw1 = ngw1; sc1 = nsc1; rb1 = nrb1;
+  }
+}
+
+static cudaError_t launch_billm_gemv(const uint16_t *X, const billm_weights *W, float *Y,
+                                     int32_t *d_status, cudaStream_t s) {
+  const size_t smem = (size_t)(W->K / 128) * (BV_STRIDE + 1) * 4 + 8 * (W->K / 128);
+  static cudaError_t attr = cudaFuncSetAttribute(
+      k_billm_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BG_SMEM_MAX);
+  if (attr != cudaSuccess) return attr;
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_billm_gemv, BG_THREADS, smem) !=
+          cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int64_t blocks =
+      std::min<int64_t>(ceil_div<int64_t>(W->N, BG_WARPS), (int64_t)sms * per_sm);
+  return launch_pdl(k_billm_gemv, dim3((unsigned)blocks), dim3(BG_THREADS), smem, s, X, W->sign,
+                    W->gmap, W->res, W->sal, W->bscale, W->N, W->K, W->ldw_words, (int)W->n_sal,
+                    Y, d_status);
+}
+
 int billm_gemm_mt(int64_t K) {
   const int64_t per = K * 4;
   int mt = BG_MT;
@@ -310,6 +451,8 @@ cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const b
     const cudaError_t e = launch_billm_gemm_tc(X, M, ldX, W, Y, ldY, d_status, s);
     if (e != cudaErrorNotSupported) return e;
   }
+  if (M == 1 && (size_t)(W->K / 128) * (BV_STRIDE + 1) * 4 + 8 * (W->K / 128) <= BG_SMEM_MAX)
+    return launch_billm_gemv(X, W, Y, d_status, s);
   const int mt = billm_gemm_mt(W->K);
   if (mt >= 4 && M >= 4) return launch_bg_t<4>(X, M, ldX, W, Y, ldY, d_status, s);
   if (mt >= 2 && M >= 2) return launch_bg_t<2>(X, M, ldX, W, Y, ldY, d_status, s);
