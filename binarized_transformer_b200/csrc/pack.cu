@@ -10,7 +10,8 @@
 namespace bwta {
 
 // ============================================================ weights (K0)
-// One warp owns a strip of 32 rows and walks K in tiles of 32 columns. Lane j
+// One warp owns a strip of 32 rows and one scale group (grid y), and walks the
+// group's columns in tiles of 32. Lane j
 // loads column j of the 32 rows (32 coalesced 128-byte loads); a ballot per
 // row yields that row's sign word. The scale needs sum|w| in ascending column
 // order (fp64), so the tile is transposed through shared memory and lane r
@@ -30,11 +31,15 @@ k_pack_weights(const float *__restrict__ W, int64_t N, int64_t K, int64_t ldW, i
   if (row0 >= N) return;
   const int64_t my_row = row0 + lane;
   const bool my_valid = my_row < N;
+  // blockIdx.y = the scale group this warp sums (its words only; the last
+  // group also writes the zero padding words up to ldw). Group sizes are
+  // multiples of 128 columns, so a group starts on a 4-word store boundary.
   double sum = 0.0;
-  int64_t g = 0, g_end = gs < K ? gs : K;  // current group and its end column
+  int64_t g = blockIdx.y, g_end = (g + 1) * gs < K ? (g + 1) * gs : K;  // group and its end column
+  const int64_t w_stop = (g == G - 1) ? ldw : (g + 1) * gs / 32;
   uint32_t words[4];
   bool bad = false;
-  for (int64_t w = 0; w < ldw; ++w) {
+  for (int64_t w = g * gs / 32; w < w_stop; ++w) {
     const int64_t k = w * 32 + lane;
     uint32_t my_word = 0;
     if (w * 32 < K) {
@@ -82,7 +87,7 @@ cudaError_t launch_pack_weights(const float *W, int64_t N, int64_t K, int64_t ld
   const int64_t G = ceil_div(K, gs);
   const int64_t warps = ceil_div<int64_t>(N, 32);
   const int64_t blocks = ceil_div<int64_t>(warps, PW_WARPS);
-  return launch_pdl(k_pack_weights, dim3((unsigned)blocks), dim3(PW_WARPS * 32), 0, s, W, N, K, ldW,
+  return launch_pdl(k_pack_weights, dim3((unsigned)blocks, (unsigned)G), dim3(PW_WARPS * 32), 0, s, W, N, K, ldW,
                     gs, G, wbits, ldw, wscale, d_status);
 }
 

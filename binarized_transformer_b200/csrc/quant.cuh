@@ -7,6 +7,8 @@
 // |x| > 0.5*mean|x|, decided exactly on integer magnitudes (units of 2^-24).
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace bwta {
@@ -47,16 +49,26 @@ __device__ __forceinline__ uint4 load_half8(const uint16_t *row, int64_t k0, int
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Exact sum of 8 fp16 magnitudes in units of 2^-24. Every finite fp16 value
+// is a multiple of 2^-24 below 2^16, so a sum of 8 needs at most 19 + 24 = 43
+// significant bits: its fp64 sum is exact in any order, and so is its product
+// with 2^24 and the conversion to an integer (the same value as the sum of
+// mag_units of the 8 patterns, for one conversion and one add per element).
+__device__ __forceinline__ double half_mag(uint32_t hm) {
+  return (double)__half2float(__ushort_as_half((unsigned short)hm));
+}
+__device__ __forceinline__ uint64_t units_of(double d) { return (uint64_t)(d * 16777216.0); }
+
 __device__ __forceinline__ uint64_t sum_mag8(const uint4 &v, bool &bad) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint64_t s = 0;
+  double d = 0.0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t hm = (w[i >> 1] >> (16 * (i & 1))) & 0x7FFFu;
     bad |= hm >= 0x7C00u;
-    s += mag_units(hm);
+    d += half_mag(hm < 0x7C00u ? hm : 0u);
   }
-  return s;
+  return units_of(d);
 }
 
 // keep / sign bit patterns of 8 halves, plus the sum of the kept magnitudes.
@@ -66,6 +78,7 @@ __device__ __forceinline__ void keep8(const uint4 &v, uint32_t hT, int64_t k0, i
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   kb = 0;
   sb = 0;
+  double kd = 0.0;  // kept magnitudes: exact, as in sum_mag8
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t h = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
@@ -73,7 +86,7 @@ __device__ __forceinline__ void keep8(const uint4 &v, uint32_t hT, int64_t k0, i
     uint32_t keep;
     if (TERNARY) {
       keep = hm > hT;
-      if (keep) ks += mag_units(hm);
+      kd += keep && hm < 0x7C00u ? half_mag(hm) : 0.0;
     } else {
       keep = (k0 + i) < K;
     }
@@ -81,6 +94,7 @@ __device__ __forceinline__ void keep8(const uint4 &v, uint32_t hT, int64_t k0, i
     kb |= keep << i;
     sb |= neg << i;
   }
+  if (TERNARY) ks += units_of(kd);
 }
 
 // E4M3 word k (k = 0..7) of a 32-element block in the tensor-core order: its
