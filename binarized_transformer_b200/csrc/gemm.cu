@@ -140,7 +140,13 @@ k_gemm_tiled(const __grid_constant__ CUtensorMap map_am, const __grid_constant__
     const int st = kt % GM_STAGES;
     const bool ok = mbar_wait(&full[st], (kt / GM_STAGES) & 1);
     if (!__syncthreads_and(ok)) {
-      if (tid == 0) flag_status(d_status, BWTA_STATUS_TIMEOUT);
+      if (tid == 0) {
+        flag_status(d_status, BWTA_STATUS_TIMEOUT);
+        // let the loads this CTA issued and has not consumed land before it exits
+        for (int j = kt; j < KT && j < kt + GM_STAGES; ++j)
+          mbar_wait(&full[j % GM_STAGES], (j / GM_STAGES) & 1, 100000000ull);
+      }
+      __syncthreads();
       return;
     }
     const uint8_t *Am = tile(st, 0), *As = tile(st, 1), *Wt = tile(st, 2);
