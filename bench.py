@@ -309,14 +309,35 @@ class LlamaStep:
         return sum(y.numel() * y.element_size() for p in self.Y_host for y in self.Y_host[p])
 
     def run_e2e(self):
-        """Host fp16 activations in, host fp32 outputs out, through the public API."""
+        """Host fp16 activations in, host fp32 outputs out, through the public API.
+        Per (phase, shape) the upload, the pack + GEMM launches and the download
+        run on three streams, ordered by events, so the two copy directions
+        overlap each other and the kernels of the neighbouring shapes. The step
+        starts after, and ends before, everything on the calling stream."""
+        comp = torch.cuda.current_stream()
+        if getattr(self, "_up", None) is None:
+            self._up, self._down = torch.cuda.Stream(), torch.cuda.Stream()
+            n = 2 * len(self.shapes)
+            self._ev_in = [torch.cuda.Event() for _ in range(n)]
+            self._ev_out = [torch.cuda.Event() for _ in range(n)]
+        self._up.wait_stream(comp)      # device inputs are free again
+        self._down.wait_stream(comp)
+        launches = self.launches()
+        i = 0
         for p in ("decode", "prefill"):
             for s in range(len(self.shapes)):
-                self.X[p][s].copy_(self.X_host[p][s], non_blocking=True)
-        self.run()
-        for p in ("decode", "prefill"):
-            for s in range(len(self.shapes)):
-                self.Y_host[p][s].copy_(self.Y[p][s], non_blocking=True)
+                with torch.cuda.stream(self._up):
+                    self.X[p][s].copy_(self.X_host[p][s], non_blocking=True)
+                    self._ev_in[i].record(self._up)
+                comp.wait_event(self._ev_in[i])
+                launches[2 * i][1]()
+                launches[2 * i + 1][1]()
+                self._ev_out[i].record(comp)
+                with torch.cuda.stream(self._down):
+                    self._down.wait_event(self._ev_out[i])
+                    self.Y_host[p][s].copy_(self.Y[p][s], non_blocking=True)
+                i += 1
+        comp.wait_stream(self._down)    # the step ends when the last output is on the host
 
 
 def capture_graph(fn):
