@@ -110,7 +110,7 @@ def tc_traffic():
 
 class ClockSampler:
     """SM clock, power and clock-event (throttle) reasons sampled while the
-    timed region runs: NVML polled from a thread every few milliseconds (the
+    timed region runs: NVML polled from a thread every 2 ms (the
     region can be far shorter than nvidia-smi's sampling period), falling back
     to `nvidia-smi -lms 50`. Read-only queries: no setting is changed."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -120,7 +120,7 @@ class ClockSampler:
     BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
             "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, cuda_index: int, interval: float = 0.005):
+    def __init__(self, cuda_index: int, interval: float = 0.002):
         self.cuda_index = cuda_index
         self.interval = interval
         self.samples = []   # (sm_mhz, power_w, reason_bits)
@@ -289,9 +289,13 @@ class LlamaStep:
                             lambda X=X, o=(m, sg, sc): bt.bwta_quantize_pack_acts(X, out=o),
                             0, qa_bytes))
                 gm_bytes = N * ld * 4 + N * G * 4 + 2 * M * ld * 4 + M * 4 + M * N * 4
+                # the weights are packed once, before any step: the decode GEMV may
+                # prefetch them before waiting for the activation pack it follows
+                flags = bt.GEMM_WEIGHTS_READY if phase == "decode" else 0
                 out.append((f"{'gemv' if phase == 'decode' else 'gemm'}_{K}x{N}_M{M}",
-                            lambda m=m, sg=sg, sc=sc, wb=wb, ws=ws, K=K, Y=Y:
-                            bt.bwta_gemm(m, sg, sc, wb, ws, K, self.group, out=(Y, None)),
+                            lambda m=m, sg=sg, sc=sc, wb=wb, ws=ws, K=K, Y=Y, flags=flags:
+                            bt.bwta_gemm(m, sg, sc, wb, ws, K, self.group, out=(Y, None),
+                                         flags=flags),
                             2 * M * N * K, gm_bytes))
         return out
 
