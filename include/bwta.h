@@ -236,13 +236,19 @@ typedef struct billm_weights {
 int billm_pack_weights(const float *W, int64_t ldW, int split, const billm_weights *out,
                        int32_t *d_status, bwta_stream_t stream);
 
-/* BiLLM-format GEMM: Y[m][n] = sum_k x[m][k] * what[n][k] with fp32
- * accumulation, evaluated per block as
+/* BiLLM-format GEMM (BiLLM abstract and "Approach": salient columns with a
+ * residual plane, non-salient weights in two groups with their own scales):
+ * Y[m][n] = sum_k x[m][k] * what[n][k], the same real value as the per-block form
  *   alpha_c*sum_C b x + alpha_sp*sum_S b x + alpha1*sum_sal b1 x + alpha2*sum_sal b2 x.
+ *  M = 1 (or X not 16-byte aligned / ldX % 8 != 0): CUDA cores, per-block sums in
+ *  fp32. M >= 2: tensor cores; each weight is rebuilt as what * 2^E (E per weight
+ *  row) split into fp16 hi + lo, and X*hi + X*lo accumulates in fp32 over all of
+ *  K. Either way |Y - Y_exact| <= 1e-5 * sum_k |x_k what_k| on finite inputs.
  *  X   fp16 bits [M][ldX]
  *  W   host pointer to a billm_weights whose buffers are device memory
  *  Y   fp32 [M][ldY] out
- *  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; NONFINITE flag. */
+ *  Errors: INVALID_ARG, UNSUPPORTED (K > 40960), ALIGNMENT, CUDA; NONFINITE and
+ *  TIMEOUT flags. */
 int billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W, float *Y,
                int64_t ldY, int32_t *d_status, bwta_stream_t stream);
 
