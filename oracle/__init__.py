@@ -53,6 +53,7 @@ def lib():
         _lib.orc_int_dots.argtypes = [vp, i64, vp, i64, i64, i64, vp]
         _lib.orc_linear_out.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
         _lib.orc_attn_scores.argtypes = [vp, vp, i64, i64, i64, i64, vp, vp, vp, vp, vp]
+        _lib.orc_softmax_ternarize.argtypes = [vp, i64, i64, C.c_float, vp, vp, vp]
         _lib.orc_billm_salient.argtypes = [vp, i64, i64, i64, i64, i64, vp]
         _lib.orc_billm_quantize_rows.argtypes = [vp, i64, i64, i64, i64, i64, i64, ip, vp, vp, vp,
                                                  vp, vp]
@@ -165,6 +166,29 @@ def attn_scores(q, k, sq, sk):
     _check(lib().orc_attn_scores(_p(q), _p(k), BH, Lq, Lk, D, _p(sq), _p(sk), _p(S), _p(fref),
                                  _p(frep)), "attn_scores")
     return S, fref, frep
+
+
+def softmax_ternarize(f, c):
+    """fp32 scores f [..., L], softmax factor c -> (a int8 {0,1} [..., L],
+    scale fp32 [...], p fp64 [..., L]): softmax of f*c per row, kept where
+    p > 1/(2L) (0.5 x the row mean), scale = mean of the kept p."""
+    f = np.ascontiguousarray(f, np.float32)
+    shape = f.shape
+    L = shape[-1]
+    R = f.size // L
+    a = np.zeros(shape, np.int8)
+    s = np.zeros(shape[:-1], np.float32)
+    p = np.zeros(shape, np.float64)
+    _check(lib().orc_softmax_ternarize(_p(f), R, L, C.c_float(c), _p(a), _p(s), _p(p)),
+           "softmax_ternarize")
+    return a, s, p
+
+
+def attn_av(a_p, s_p, a_vt, s_vt):
+    """A . V with ternary probabilities a_p [BH, Lq, L] (scales s_p [BH, Lq])
+    and ternary V^T rows a_vt [BH, D, L] (scales s_vt [BH, D]) ->
+    (O int64, O fp64, O fp32 replica), each [BH, Lq, D]."""
+    return attn_scores(a_p, a_vt, s_p, s_vt)
 
 
 def billm_salient(W, block=128, n_sal=8):

@@ -258,6 +258,53 @@ int orc_attn_scores(const int8_t *q, const int8_t *k, int64_t BH, int64_t Lq, in
   return ORC_OK;
 }
 
+/* ------------------------------------------ attention probabilities, A.V
+ * [BWTA] abstract: the binary/ternary MatMul serves the attention operators,
+ * so the attention probabilities, the activations that enter A . V, are
+ * ternarized like any activation (reading R17): keep p iff p > 0.5 * mean(p)
+ * over the row. A softmax row sums to 1, so its mean is exactly 1/L and the
+ * test reads p > 1/(2L); every p is positive, so a kept value is +1. The row
+ * scale is the mean of the kept p (0 if none).
+ * Input: f fp32 [R][L], the scores of one query row each (the fp32 output of
+ * the Q . K^T product), and the softmax factor c; x = f * c in fp32.
+ * p = exp(x - max x) / sum exp(x - max x), in fp64 (exp of the math library).
+ * Output: a int8 [R][L] in {0, 1}; scale fp32 [R] (fp64 sum of the kept p in
+ * ascending column order, divided by the count, rounded once); p fp64 [R][L]
+ * (may be NULL).
+ * A . V itself is orc_attn_scores with the ternary probabilities as the query
+ * side and the rows of V^T (one per output channel, ternarized over the
+ * sequence) as the key side: the contraction runs over the L keys.
+ */
+int orc_softmax_ternarize(const float *f, int64_t R, int64_t L, float c, int8_t *a, float *scale,
+                          double *p_out) {
+  if (R < 0 || L <= 0) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < R; ++r) {
+    const float *fr = f + r * L;
+    double mx = -INFINITY;
+    for (int64_t j = 0; j < L; ++j) {
+      const float x = fr[j] * c;
+      if ((double)x > mx) mx = (double)x;
+    }
+    double z = 0.0;
+    for (int64_t j = 0; j < L; ++j) z += exp((double)(fr[j] * c) - mx);
+    double kept = 0.0;
+    int64_t n = 0;
+    for (int64_t j = 0; j < L; ++j) {
+      const double p = exp((double)(fr[j] * c) - mx) / z;
+      if (p_out) p_out[r * L + j] = p;
+      const int keep = p > 0.5 / (double)L;
+      a[r * L + j] = (int8_t)keep;
+      if (keep) {
+        kept += p;
+        ++n;
+      }
+    }
+    scale[r] = n ? (float)(kept / (double)n) : 0.0f;
+  }
+  return ORC_OK;
+}
+
 /* ------------------------------------------------------- BiLLM quantizer
  * Salient columns ([BiLLM] Approach, reading R4): per block of `block`
  * columns, the n_sal columns with the largest sum_n w^2 (fp64, n ascending);

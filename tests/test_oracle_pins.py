@@ -321,3 +321,60 @@ def test_billm_pack_matches_numpy_packbits(orc):
         b2s = q["b2"][:, j * 128 + sal[j]] < 0
         np.testing.assert_array_equal(p["res"][:, j], np.packbits(b2s, axis=1, bitorder="little")[:, 0])
         np.testing.assert_array_equal(p["sal"][j], sal[j])
+
+
+# ------------------------------------------------ attention probabilities, A.V
+def _golden_scores(tok):
+    return float(np.log(float(tok[2:]))) if tok.startswith("ln") else float(tok)
+
+
+def test_softmax_ternarize_golden_rows(orc):
+    for scores, c, keep, scale in read_golden("softmax_rows.txt"):
+        f = np.array([[_golden_scores(t) for t in scores.split()]], np.float32)
+        a, s, p = orc.softmax_ternarize(f, float(c))
+        assert a[0].tolist() == [int(t) for t in keep.split()], scores
+        assert abs(float(s[0]) - float(scale)) <= 1e-6 * float(scale), (scores, s)
+        assert abs(p.sum() - 1.0) < 1e-12
+
+
+def test_softmax_ternarize_matches_numpy(orc):
+    g = np.random.default_rng(42)
+    f = (g.standard_normal((64, 300)) * 3).astype(np.float32)
+    c = 0.125
+    a, s, p = orc.softmax_ternarize(f, c)
+    x = (f * np.float32(c)).astype(np.float64)       # the product in fp32, as the definition
+    e = np.exp(x - x.max(axis=1, keepdims=True))
+    pn = e / e.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(p, pn, rtol=1e-13, atol=0)
+    keep = pn > 0.5 / f.shape[1]
+    np.testing.assert_array_equal(a.astype(bool), keep)
+    mean_kept = np.array([pn[r, keep[r]].mean() if keep[r].any() else 0.0 for r in range(64)])
+    np.testing.assert_array_equal(s, mean_kept.astype(np.float32))
+
+
+def test_softmax_ternarize_invariants(orc):
+    g = np.random.default_rng(7)
+    f = g.integers(-20, 20, (16, 128)).astype(np.float32)
+    a, s, p = orc.softmax_ternarize(f, 0.5)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    a2, s2, p2 = orc.softmax_ternarize(f + 6.0, 0.5)   # a shift of the row (exact in fp32)
+    np.testing.assert_array_equal(a, a2)
+    np.testing.assert_allclose(p2, p, rtol=1e-12)
+    assert ((a == 0) | (a == 1)).all() and (a.sum(axis=1) >= 1).all()   # the max is always kept
+
+
+def test_attn_av_matches_dense_dequantized_product(orc):
+    g = np.random.default_rng(3)
+    BH, Lq, L, D = 2, 5, 96, 7
+    f = (g.standard_normal((BH, Lq, L)) * 4).astype(np.float32)
+    ap, sp, _ = orc.softmax_ternarize(f, 0.25)
+    V = g.standard_normal((BH, L, D)).astype(np.float16)
+    vt = np.ascontiguousarray(V.transpose(0, 2, 1)).reshape(-1, L)
+    av, sv = orc.quantize_acts(vt)
+    O, Oref, Orep = orc.attn_av(ap, sp, av.reshape(BH, D, L), sv.reshape(BH, D))
+    Pd = ap.astype(np.float64) * sp[..., None].astype(np.float64)
+    Vd = av.reshape(BH, D, L).astype(np.float64) * sv.reshape(BH, D)[..., None].astype(np.float64)
+    dense = np.einsum("hql,hdl->hqd", Pd, Vd)
+    np.testing.assert_allclose(Oref, dense, rtol=1e-12, atol=1e-300)
+    np.testing.assert_array_equal(O, np.einsum("hql,hdl->hqd", ap.astype(np.int64),
+                                               av.reshape(BH, D, L).astype(np.int64)))
