@@ -210,11 +210,19 @@ class ClockSampler:
 
 
 class L2Flusher:
+    """Between timed steps: write a 256 MiB buffer (twice the 126 MB L2), then
+    read another 256 MiB buffer. The write evicts everything the last step left
+    in L2; the read replaces the flush's own dirty lines with clean ones, so the
+    timed kernels start cold and none of their reads waits behind a write-back
+    of the flush."""
+
     def __init__(self):
         self.buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.rbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
 
     def __call__(self):
         self.buf.zero_()
+        self.rbuf.sum(dtype=torch.int64)
 
 
 def event_pair():
@@ -261,13 +269,33 @@ class LlamaStep:
                 self.Y[phase].append(torch.empty((M, N), dtype=torch.float32, device="cuda"))
         self.Y_host = {p: [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in self.Y[p]]
                        for p in self.Y}
+        # the decode phase: the three projections in one fused launch
+        self.decode_desc = bt.decode_jobs([(self.X["decode"][s], self.w[s][0], self.w[s][1],
+                                            self.group, self.Y["decode"][s], None)
+                                           for s in range(len(self.shapes))])
         torch.cuda.synchronize()
+
+    def decode_launch(self):
+        """The decode phase: ternarize the three M=1 rows and run the three GEMVs
+        in one launch (weights were packed before any step, so the kernel may
+        stream them before the previous kernel in the stream has finished)."""
+        bt = self.bt
+        M = self.M["decode"]
+        ops = nbytes = 0
+        for s, (K, N) in enumerate(self.shapes):
+            ld = bt.ld_words_for(K)
+            ops += 2 * M * N * K
+            nbytes += N * ld * 4 + N * (K // self.group) * 4 + M * K * 2 + M * N * 4
+        return ("decode_batched_3_projections_M1",
+                lambda: bt.bwta_linear_decode_batched(None, flags=bt.GEMM_WEIGHTS_READY,
+                                                      descriptors=self.decode_desc),
+                ops, nbytes)
 
     def launches(self):
         """(name, callable, ops, alg_bytes) for every kernel launch of one step, in order."""
         bt = self.bt
-        out = []
-        for phase in ("decode", "prefill"):
+        out = [self.decode_launch()]
+        for phase in ("prefill",):
             for s, (K, N) in enumerate(self.shapes):
                 M = self.M[phase]
                 X, (m, sg, sc, a8), Y = self.X[phase][s], self.planes[phase][s], self.Y[phase][s]
@@ -299,6 +327,27 @@ class LlamaStep:
                             2 * M * N * K, gm_bytes))
         return out
 
+    def popc_launches(self):
+        """The prefill products on the LOP3+POPC path (bit planes + k_gemm_tiled),
+        timed beside the step so that the popcount kernel's roofline is recorded
+        in every bench line."""
+        bt = self.bt
+        out = []
+        M = self.M["prefill"]
+        for s, (K, N) in enumerate(self.shapes):
+            X, (m, sg, sc, _), Y = self.X["prefill"][s], self.planes["prefill"][s], self.Y["prefill"][s]
+            wb, ws = self.w[s]
+            ld = m.shape[1]
+            G = K // self.group
+            out.append((f"quantize_pack_planes_prefill_{K}x{N}",
+                        lambda X=X, o=(m, sg, sc): bt.bwta_quantize_pack_acts(X, out=o),
+                        0, M * K * 2 + 2 * M * ld * 4 + M * 4))
+            out.append((f"gemm_popc_{K}x{N}_M{M}",
+                        lambda m=m, sg=sg, sc=sc, wb=wb, ws=ws, K=K, Y=Y:
+                        bt.bwta_gemm(m, sg, sc, wb, ws, K, self.group, out=(Y, None)),
+                        2 * M * N * K, N * ld * 4 + N * G * 4 + 2 * M * ld * 4 + M * 4 + M * N * 4))
+        return out
+
     def ops(self):
         return sum(op for _, _, op, _ in self.launches())
 
@@ -314,33 +363,37 @@ class LlamaStep:
 
     def run_e2e(self):
         """Host fp16 activations in, host fp32 outputs out, through the public API.
-        Per (phase, shape) the upload, the pack + GEMM launches and the download
-        run on three streams, ordered by events, so the two copy directions
-        overlap each other and the kernels of the neighbouring shapes. The step
-        starts after, and ends before, everything on the calling stream."""
+        The decode phase (three rows up, one launch, three outputs down) and then
+        each prefill shape (upload, pack + GEMM, download) run on three streams,
+        ordered by events, so the two copy directions overlap each other and the
+        kernels of the neighbouring shapes. The step starts after, and ends
+        before, everything on the calling stream."""
         comp = torch.cuda.current_stream()
+        n = 1 + len(self.shapes)
         if getattr(self, "_up", None) is None:
             self._up, self._down = torch.cuda.Stream(), torch.cuda.Stream()
-            n = 2 * len(self.shapes)
             self._ev_in = [torch.cuda.Event() for _ in range(n)]
             self._ev_out = [torch.cuda.Event() for _ in range(n)]
         self._up.wait_stream(comp)      # device inputs are free again
         self._down.wait_stream(comp)
         launches = self.launches()
-        i = 0
-        for p in ("decode", "prefill"):
-            for s in range(len(self.shapes)):
-                with torch.cuda.stream(self._up):
+        # unit 0: the decode phase; units 1..3: the prefill shapes
+        units = [([("decode", s) for s in range(len(self.shapes))], [launches[0]])]
+        for s in range(len(self.shapes)):
+            units.append(([("prefill", s)], launches[1 + 2 * s:3 + 2 * s]))
+        for i, (tensors, kernels) in enumerate(units):
+            with torch.cuda.stream(self._up):
+                for p, s in tensors:
                     self.X[p][s].copy_(self.X_host[p][s], non_blocking=True)
-                    self._ev_in[i].record(self._up)
-                comp.wait_event(self._ev_in[i])
-                launches[2 * i][1]()
-                launches[2 * i + 1][1]()
-                self._ev_out[i].record(comp)
-                with torch.cuda.stream(self._down):
-                    self._down.wait_event(self._ev_out[i])
+                self._ev_in[i].record(self._up)
+            comp.wait_event(self._ev_in[i])
+            for k in kernels:
+                k[1]()
+            self._ev_out[i].record(comp)
+            with torch.cuda.stream(self._down):
+                self._down.wait_event(self._ev_out[i])
+                for p, s in tensors:
                     self.Y_host[p][s].copy_(self.Y[p][s], non_blocking=True)
-                i += 1
         comp.wait_stream(self._down)    # the step ends when the last output is on the host
 
 
@@ -385,10 +438,10 @@ def time_steps(step_fn, steps, warmup, flush):
     return total, per
 
 
-def per_kernel_times(step, reps, flush):
+def per_kernel_times(step, reps, flush, launches=None):
     """Average device time of every launch of a step, each bracketed by events
     on the launching stream (eager launches, L2 flushed before each step)."""
-    launches = step.launches()
+    launches = step.launches() if launches is None else launches
     acc = {name: [] for name, _, _, _ in launches}
     for _ in range(reps):
         flush()
@@ -459,13 +512,23 @@ def run_ours(args):
     e2e_value = weak_scaling_value(ops_step, max(1, args.steps), world, e2e_max) / 1e12
 
     kern = per_kernel_times(step, max(3, args.steps), flush)
+    # the popcount GEMMs, each timed alone (flush, GPU head start, events): the
+    # bit planes they read are packed once first
+    kern_popc = {}
+    for name, fn, ops, nbytes in step.popc_launches():
+        if name.startswith("gemm_popc"):
+            kern_popc[name] = {"s": _time_fn(fn, max(3, args.steps), flush), "ops": ops,
+                               "bytes": nbytes}
+        else:
+            fn()
 
     if rank != 0:
         barrier()
         return
     peaks, peak_src = measured_peaks()
-    wordop = mb.rate("wordop")          # word-ops / s: LOP3 + POPC + add
-    popc_peak_tops = wordop * 64 / 1e12  # one word-op = 32 MACs = 64 ops
+    # word-ops / s of the tiled kernel's own inner mix (per 4-word chunk: 6 LOP3,
+    # 3 POPC, adds); one word-op = 32 MACs = 64 ops
+    popc_peak_tops = mb.rate("popc4") * 64 / 1e12
     gemms = {k: v for k, v in kern.items() if k.startswith("gemm_")}
     g_ops = sum(v["ops"] for v in gemms.values())
     g_s = sum(v["s"] for v in gemms.values())
@@ -477,7 +540,10 @@ def run_ours(args):
     fp8_src = ("2 x measured bf16 burst (MEASURED_PEAKS.json)" if "bf16_tflops" in peaks
                else "2 x fallback bf16 1590 TFLOP/s")
     kernels = {}
-    for name, v in kern.items():
+    popc_gemms = {k: v for k, v in kern_popc.items() if k.startswith("gemm_popc")}
+    p_ops = sum(v["ops"] for v in popc_gemms.values())
+    p_s = sum(v["s"] for v in popc_gemms.values())
+    for name, v in list(kern.items()) + list(kern_popc.items()):
         e = {"us": round(v["s"] * 1e6, 3), "alg_bytes": v["bytes"],
              "gbs": round(v["bytes"] / v["s"] / 1e9, 1)}
         if v["ops"]:
@@ -498,7 +564,7 @@ def run_ours(args):
         "config": {"workload": "llama7b_projections", "shapes_KxN": [list(s) for s in step.shapes],
                    "M_prefill": step.M["prefill"], "M_decode": step.M["decode"],
                    "group": step.group, "acts": "student-t(3), 1% x20 outliers, ternarized",
-                   "l2": "flushed before every step (256 MiB write)",
+                   "l2": "flushed before every step (256 MiB write, then 256 MiB read)",
                    "parallelism": f"dp{world}" if world > 1 else "single"},
         "roofline": ({"bound": "tensor", "kernel": "k_gemm_tc (prefill, 3 shapes)",
                       "achieved": round(achieved, 3), "peak": round(fp8_peak, 1),
@@ -510,8 +576,14 @@ def run_ours(args):
                      {"bound": "alu", "kernel": "k_gemm_tiled (prefill, 3 shapes)",
                       "achieved": round(achieved, 3), "peak": round(popc_peak_tops, 3),
                       "unit": "TOPS", "frac": round(achieved / popc_peak_tops, 4),
-                      "peak_source": "microbenchmarked LOP3+POPC+IADD word-op rate x 64 ops/word",
+                      "peak_source": "microbenchmarked rate of the kernel's inner mix per 4-word "
+                                     "chunk (4+2 LOP3, 3 POPC, adds) x 64 ops per word",
                       "traffic": None}),
+        "popc_roofline": {"bound": "alu", "kernel": "k_gemm_tiled (prefill, 3 shapes, timed beside the step)",
+                          "achieved": round(p_ops / p_s / 1e12, 3), "peak": round(popc_peak_tops, 3),
+                          "unit": "TOPS", "frac": round(p_ops / p_s / 1e12 / popc_peak_tops, 4),
+                          "peak_source": "microbenchmarked rate of the kernel's inner mix per 4-word "
+                                         "chunk (4+2 LOP3, 3 POPC, adds) x 64 ops per word"},
         "cpu_baseline": {"value": round(cpu_ops / cpu_s / 1e12, 6), "unit": UNIT, "cores": cores,
                          "kind": "oracle",
                          "sample": f"{args.cpu_rows} prefill rows per shape + the decode row, "
@@ -639,7 +711,7 @@ def run_rows(args):
     flush = L2Flusher()
     peaks, _ = measured_peaks()
     hbm = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
-    popc_tops = mb.rate("wordop") * 64 / 1e12
+    popc_tops = mb.rate("popc4") * 64 / 1e12
     reps = max(3, args.steps)
     rows = args.workload.split(",")
     if "all" in rows:

@@ -21,14 +21,14 @@ LIB_PATH = os.path.join(_HERE, "libbwta.so")
 MB_LIB_PATH = os.path.join(_HERE, "libbwta_microbench.so")
 
 BWTA_OK, BWTA_ERR_INVALID_ARG, BWTA_ERR_UNSUPPORTED, BWTA_ERR_ALIGNMENT, BWTA_ERR_CUDA = range(5)
-STATUS_NONFINITE, STATUS_TIMEOUT = 0x1, 0x2
+STATUS_NONFINITE, STATUS_TIMEOUT, STATUS_DRAIN = 0x1, 0x2, 0x4
 TERNARY, BINARY = 0, 1
 ERROR_NAMES = {1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA"}
 
 EXPORTS = ["bwta_pack_weights", "bwta_quantize_pack_acts", "bwta_quantize_pack_acts_ex",
            "bwta_gemm", "bwta_gemm_ex", "bwta_gemm_tc",
            "bwta_linear_decode", "bwta_attn_scores", "billm_pack_weights", "billm_gemm",
-           "bwta_version"]
+           "bwta_linear_decode_batched", "bwta_selftest_gemm_timeout", "bwta_version"]
 GEMM_WEIGHTS_READY = 0x1
 
 
@@ -43,6 +43,13 @@ class BillmWeightsC(C.Structure):
                 ("sal", C.c_void_p), ("bscale", C.c_void_p), ("N", C.c_int64),
                 ("K", C.c_int64), ("ldw_words", C.c_int64), ("block", C.c_int64),
                 ("n_sal", C.c_int64)]
+
+
+class DecodeJobC(C.Structure):
+    _fields_ = [("X", C.c_void_p), ("M", C.c_int64), ("K", C.c_int64), ("ldX", C.c_int64),
+                ("wbits", C.c_void_p), ("wscale", C.c_void_p), ("N", C.c_int64),
+                ("ldw_words", C.c_int64), ("group", C.c_int64), ("Y", C.c_void_p),
+                ("ldY", C.c_int64), ("dots", C.c_void_p), ("ldD", C.c_int64)]
 
 
 _lib = None
@@ -72,6 +79,10 @@ def load_library(path: str = LIB_PATH):
     lib.bwta_attn_scores.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp, vp]
     lib.billm_pack_weights.argtypes = [vp, i64, ci, C.POINTER(BillmWeightsC), vp, vp]
     lib.billm_gemm.argtypes = [vp, i64, i64, C.POINTER(BillmWeightsC), vp, i64, vp, vp]
+    lib.bwta_linear_decode_batched.argtypes = [C.POINTER(DecodeJobC), i64, ci, cf, C.c_uint32, vp,
+                                               vp]
+    lib.bwta_selftest_gemm_timeout.argtypes = [vp, vp, vp, i64, i64, vp, vp, i64, i64, i64, i64,
+                                               vp, i64, vp, i64, i64, vp, vp]
     lib.bwta_version.restype = C.c_char_p
     for name in EXPORTS[:-1]:
         getattr(lib, name).restype = C.c_int
@@ -223,6 +234,26 @@ def bwta_gemm(a_mask, a_sign, a_scale, wbits, wscale, K: int, group: int = 0,
     return Y, D
 
 
+def bwta_selftest_gemm_timeout(a_mask, a_sign, a_scale, wbits, wscale, K: int, group: int = 0,
+                               wait_limit_ns: int = 1_000_000, status=None, out=None):
+    """Failure-path self-test: the tiled GEMM with a wait that is made to run
+    out after wait_limit_ns. Returns the status tensor (BWTA_STATUS_TIMEOUT set)."""
+    lib = _L()
+    M, lda = a_mask.shape
+    N, ldw = wbits.shape
+    status = new_status(a_mask.device) if status is None else status
+    if out is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=a_mask.device)
+        D = None
+    else:
+        Y, D = out
+    _check("bwta_selftest_gemm_timeout", lib.bwta_selftest_gemm_timeout(
+        _ptr(a_mask), _ptr(a_sign), _ptr(a_scale), M, lda, _ptr(wbits), _ptr(wscale), N, ldw, K,
+        group, _ptr(Y), _row_stride(Y) if Y is not None else N, _ptr(D),
+        _row_stride(D) if D is not None else N, wait_limit_ns, _ptr(status), _stream()))
+    return status
+
+
 def bwta_linear_decode(X, wbits, wscale, group: int = 0, mode: int = TERNARY,
                        thresh_ratio: float = 0.5, want_y: bool = True, want_dots: bool = False,
                        flags: int = 0, status=None, out=None):
@@ -242,6 +273,45 @@ def bwta_linear_decode(X, wbits, wscale, group: int = 0, mode: int = TERNARY,
         _ptr(Y), _row_stride(Y) if Y is not None else N, _ptr(D),
         _row_stride(D) if D is not None else N, flags, _ptr(status), _stream()))
     return Y, D
+
+
+def decode_jobs(jobs, want_dots: bool = False):
+    """C descriptors for bwta_linear_decode_batched. Each job is a tuple
+    (X fp16 [M, K], wbits, wscale, group) or (X, wbits, wscale, group, Y, dots)
+    with preallocated outputs (either may be None). Returns (array, outputs)."""
+    arr = (DecodeJobC * max(1, len(jobs)))()
+    outs = []
+    for i, job in enumerate(jobs):
+        X, wbits, wscale, group = job[:4]
+        assert X.is_cuda and X.dtype == torch.float16 and X.dim() == 2 and X.stride(1) == 1
+        M, K = X.shape
+        N, ldw = wbits.shape
+        if len(job) > 4:
+            Y, D = job[4], job[5]
+        else:
+            Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+            D = torch.empty((M, N), dtype=torch.int32, device=X.device) if want_dots else None
+        arr[i] = DecodeJobC(X.data_ptr(), M, K, _row_stride(X), wbits.data_ptr(), wscale.data_ptr(),
+                            N, ldw, group, Y.data_ptr() if Y is not None else None,
+                            _row_stride(Y) if Y is not None else N,
+                            D.data_ptr() if D is not None else None,
+                            _row_stride(D) if D is not None else N)
+        outs.append((Y, D))
+    return arr, outs
+
+
+def bwta_linear_decode_batched(jobs, mode: int = TERNARY, thresh_ratio: float = 0.5,
+                               want_dots: bool = False, flags: int = 0, status=None,
+                               descriptors=None):
+    """Several fused decode projections in one launch. `jobs` as decode_jobs();
+    or pass `descriptors` = decode_jobs(...) built once (the outputs they name).
+    Returns [(Y, dots or None)] per job."""
+    lib = _L()
+    arr, outs = descriptors if descriptors is not None else decode_jobs(jobs, want_dots)
+    n = len(outs)
+    _check("bwta_linear_decode_batched", lib.bwta_linear_decode_batched(
+        arr, n, mode, thresh_ratio, flags, _ptr(status), _stream()))
+    return outs
 
 
 def bwta_attn_scores(q_mask, q_sign, q_scale, k_mask, k_sign, k_scale, BH: int, Lq: int, Lk: int,

@@ -25,7 +25,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
                 "-I", os.path.join(ROOT, "include")]
 
-LIB_SOURCES = ["pack.cu", "gemm.cu", "gemm_tc.cu", "attn.cu", "billm.cu", "billm_tc.cu", "abi.cu"]
+LIB_SOURCES = ["pack.cu", "gemm.cu", "decode.cu", "gemm_tc.cu", "attn.cu", "billm.cu", "billm_tc.cu",
+               "abi.cu"]
 MB_SOURCES = ["microbench.cu"]
 HEADERS = ["common.cuh", "tma.cuh", "quant.cuh", "tcgen05.cuh"]
 

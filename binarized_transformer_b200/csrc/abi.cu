@@ -131,34 +131,115 @@ int bwta_gemm_ex(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_
   if (int r = check_plane(wbits, N, ldw_words, K)) return r;
   if (M == 0 || N == 0) return BWTA_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  if (gemv_fits(M, lda_words, K, group))
-    return cuda_status(launch_gemv(a_mask, a_sign, a_scale, M, lda_words, wbits, wscale, N,
-                                   ldw_words, K, group, Y, ldY, dots, ldD,
-                                   (flags & BWTA_GEMM_WEIGHTS_READY) != 0, s));
+  if (decode_fits(M, K)) {
+    DecodeSpec job = {};
+    job.am = a_mask;
+    job.as = a_sign;
+    job.ascale = a_scale;
+    job.lda = lda_words;
+    job.M = M;
+    job.K = K;
+    job.wbits = wbits;
+    job.wscale = wscale;
+    job.N = N;
+    job.ldw = ldw_words;
+    job.group = group;
+    job.Y = Y;
+    job.ldY = ldY;
+    job.dots = dots;
+    job.ldD = ldD;
+    return cuda_status(launch_decode(&job, 1, false, BWTA_TERNARY,
+                                     (flags & BWTA_GEMM_WEIGHTS_READY) != 0, d_status, s));
+  }
   return cuda_status(launch_gemm_tiled(a_mask, a_sign, a_scale, M, lda_words, wbits, wscale, N,
-                                       ldw_words, K, group, Y, ldY, dots, ldD, d_status, s));
+                                       ldw_words, K, group, Y, ldY, dots, ldD, d_status, 0, s));
+}
+
+int bwta_selftest_gemm_timeout(const uint32_t *a_mask, const uint32_t *a_sign,
+                               const float *a_scale, int64_t M, int64_t lda_words,
+                               const uint32_t *wbits, const float *wscale, int64_t N,
+                               int64_t ldw_words, int64_t K, int64_t group, float *Y, int64_t ldY,
+                               int32_t *dots, int64_t ldD, int64_t wait_limit_ns,
+                               int32_t *d_status, bwta_stream_t stream) {
+  if (!d_status || M <= 8 || wait_limit_ns < 1 || wait_limit_ns > 2000000000LL)
+    return BWTA_ERR_INVALID_ARG;
+  if (N < 0 || K <= 0) return BWTA_ERR_INVALID_ARG;
+  if (K > BWTA_MAX_K) return BWTA_ERR_UNSUPPORTED;
+  if (int r = check_group(group)) return r;
+  if (!Y && !dots) return BWTA_ERR_INVALID_ARG;
+  if (Y && ldY < N) return BWTA_ERR_INVALID_ARG;
+  if (dots && ldD < N) return BWTA_ERR_INVALID_ARG;
+  if (!a_scale || (N > 0 && !wscale)) return BWTA_ERR_INVALID_ARG;
+  if (int r = check_plane(a_mask, M, lda_words, K)) return r;
+  if (int r = check_plane(a_sign, M, lda_words, K)) return r;
+  if (int r = check_plane(wbits, N, ldw_words, K)) return r;
+  if (N == 0) return BWTA_OK;
+  return cuda_status(launch_gemm_tiled(a_mask, a_sign, a_scale, M, lda_words, wbits, wscale, N,
+                                       ldw_words, K, group, Y, ldY, dots, ldD, d_status,
+                                       (uint64_t)wait_limit_ns, (cudaStream_t)stream));
+}
+
+// Validation shared by the single and the batched fused decode.
+static int check_decode_job(const bwta_decode_job &J) {
+  if (J.M < 0 || J.N < 0 || J.K <= 0 || J.ldX < J.K) return BWTA_ERR_INVALID_ARG;
+  if (J.M > 8 || !decode_fits(J.M > 0 ? J.M : 1, J.K)) return BWTA_ERR_UNSUPPORTED;
+  if (int r = check_group(J.group)) return r;
+  if (J.M > 0 && J.N > 0 && !J.Y && !J.dots) return BWTA_ERR_INVALID_ARG;
+  if (J.Y && J.ldY < J.N) return BWTA_ERR_INVALID_ARG;
+  if (J.dots && J.ldD < J.N) return BWTA_ERR_INVALID_ARG;
+  if (J.M > 0 && !J.X) return BWTA_ERR_INVALID_ARG;
+  if (J.N > 0 && !J.wscale) return BWTA_ERR_INVALID_ARG;
+  if (int r = check_plane(J.wbits, J.N, J.ldw_words, J.K)) return r;
+  return BWTA_OK;
+}
+
+static DecodeSpec fused_spec(const bwta_decode_job &J) {
+  DecodeSpec d = {};
+  d.X = J.X;
+  d.ldX = J.ldX;
+  d.M = J.M;
+  d.K = J.K;
+  d.wbits = J.wbits;
+  d.wscale = J.wscale;
+  d.N = J.N;
+  d.ldw = J.ldw_words;
+  d.group = J.group;
+  d.Y = J.Y;
+  d.ldY = J.ldY;
+  d.dots = J.dots;
+  d.ldD = J.ldD;
+  return d;
 }
 
 int bwta_linear_decode(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
                        float thresh_ratio, const uint32_t *wbits, const float *wscale, int64_t N,
                        int64_t ldw_words, int64_t group, float *Y, int64_t ldY, int32_t *dots,
                        int64_t ldD, uint32_t flags, int32_t *d_status, bwta_stream_t stream) {
+  const bwta_decode_job J = {X, M, K, ldX, wbits, wscale, N, ldw_words, group, Y, ldY, dots, ldD};
+  return bwta_linear_decode_batched(&J, 1, mode, thresh_ratio, flags, d_status, stream);
+}
+
+int bwta_linear_decode_batched(const bwta_decode_job *jobs, int64_t njobs, int mode,
+                               float thresh_ratio, uint32_t flags, int32_t *d_status,
+                               bwta_stream_t stream) {
   if (flags & ~BWTA_GEMM_WEIGHTS_READY) return BWTA_ERR_INVALID_ARG;
-  if (M < 0 || N < 0 || K <= 0 || ldX < K) return BWTA_ERR_INVALID_ARG;
+  if (njobs < 0 || (njobs > 0 && !jobs)) return BWTA_ERR_INVALID_ARG;
+  if (njobs > decode_max_jobs()) return BWTA_ERR_UNSUPPORTED;
   if (mode != BWTA_TERNARY && mode != BWTA_BINARY) return BWTA_ERR_INVALID_ARG;
   if (thresh_ratio != 0.5f) return BWTA_ERR_UNSUPPORTED;
-  if (M > 8 || !linear_decode_fits(M > 0 ? M : 1, K)) return BWTA_ERR_UNSUPPORTED;
-  if (int r = check_group(group)) return r;
-  if (!Y && !dots) return BWTA_ERR_INVALID_ARG;
-  if (Y && ldY < N) return BWTA_ERR_INVALID_ARG;
-  if (dots && ldD < N) return BWTA_ERR_INVALID_ARG;
-  if (M > 0 && !X) return BWTA_ERR_INVALID_ARG;
-  if (N > 0 && !wscale) return BWTA_ERR_INVALID_ARG;
-  if (int r = check_plane(wbits, N, ldw_words, K)) return r;
-  if (M == 0 || N == 0) return BWTA_OK;
-  return cuda_status(launch_linear_decode(X, M, K, ldX, mode, wbits, wscale, N, ldw_words, group,
-                                          Y, ldY, dots, ldD, (flags & BWTA_GEMM_WEIGHTS_READY) != 0,
-                                          d_status, (cudaStream_t)stream));
+  DecodeSpec spec[8];
+  size_t act = 0;
+  int n = 0;
+  for (int64_t i = 0; i < njobs; ++i) {
+    if (int r = check_decode_job(jobs[i])) return r;
+    if (jobs[i].M == 0 || jobs[i].N == 0) continue;
+    act += decode_act_bytes(jobs[i].M, jobs[i].K);
+    spec[n++] = fused_spec(jobs[i]);
+  }
+  if (act > decode_max_act_bytes()) return BWTA_ERR_UNSUPPORTED;
+  if (n == 0) return BWTA_OK;
+  return cuda_status(launch_decode(spec, n, true, mode, (flags & BWTA_GEMM_WEIGHTS_READY) != 0,
+                                   d_status, (cudaStream_t)stream));
 }
 
 int bwta_attn_scores(const uint32_t *q_mask, const uint32_t *q_sign, const float *q_scale,

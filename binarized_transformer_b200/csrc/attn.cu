@@ -188,6 +188,148 @@ static cudaError_t launch_attn_nw(const uint32_t *qm, const uint32_t *qs, const 
 #undef BWTA_AT
 }
 
+// ============================================ softmax -> ternary probabilities
+// The attention probabilities are the activations of the A . V product, so
+// they are ternarized like any activation (BWTA abstract: binary/ternary
+// MatMul for the attention operators): keep p iff p > 0.5 * mean(p) over the
+// row. A softmax row sums to one, so that threshold is 1/(2 Lk); every p is
+// positive, so the kept values are +1 (the sign plane is all zero) and the row
+// scale is the mean of the kept p. This kernel goes from the ternary Q and K
+// planes straight to those planes: the Lq x Lk scores are never written to
+// memory. One CTA per (batch*head, 64 query rows) holds the head's K planes in
+// shared memory; a warp owns a query row: per key, the ternary dot, the fp32
+// score ((float)S * s_q) * s_k (the same value bwta_attn_scores writes) times
+// the softmax factor; then the row max, e = exp(x - max), the sum, p = e / sum,
+// the keep bits (one ballot per 32 keys is one mask word) and the kept sum.
+constexpr int AS_ROWS = 64, AS_THREADS = 256, AS_WARPS = AS_THREADS / 32;
+
+template <int NW>
+__global__ void __launch_bounds__(AS_THREADS)
+k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict__ qs,
+                    const float *__restrict__ qscale, const uint32_t *__restrict__ km,
+                    const uint32_t *__restrict__ ks, const float *__restrict__ kscale, int64_t Lq,
+                    int64_t Lk, int ld, float c, uint32_t *__restrict__ pm, uint32_t *__restrict__ ps,
+                    int ldp, float *__restrict__ pscale) {
+  extern __shared__ uint4 as_sm[];
+  const int nc = NW == 4 ? ld / 4 : 1;
+  uint4 *sKm = as_sm;
+  uint4 *sKs = sKm + Lk * nc;
+  float *sk = reinterpret_cast<float *>(sKs + Lk * nc);
+  float *xw = sk + Lk + (threadIdx.x / 32) * Lk;  // this warp's row of scores, then of exp
+  pdl_trigger();
+  pdl_wait();
+  const int64_t bh = blockIdx.y;
+  for (int idx = threadIdx.x; idx < Lk * nc; idx += AS_THREADS) {
+    const int64_t off = (bh * Lk + idx / nc) * ld;
+    sKm[idx] = __ldg(reinterpret_cast<const uint4 *>(km + off) + idx % nc);
+    sKs[idx] = __ldg(reinterpret_cast<const uint4 *>(ks + off) + idx % nc);
+  }
+  for (int idx = threadIdx.x; idx < Lk; idx += AS_THREADS) sk[idx] = __ldg(kscale + bh * Lk + idx);
+  __syncthreads();
+
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  const float thr = 0.5f / (float)Lk;
+  for (int r = w; r < AS_ROWS; r += AS_WARPS) {
+    const int64_t i = (int64_t)blockIdx.x * AS_ROWS + r;
+    if (i >= Lq) break;
+    const int64_t qrow = (bh * Lq + i) * ld;
+    const float sqi = __ldg(qscale + bh * Lq + i);
+    uint4 qa[NW == 4 ? 8 : 1], qb[NW == 4 ? 8 : 1];
+#pragma unroll
+    for (int cc = 0; cc < (NW == 4 ? 8 : 1); ++cc) {
+      if (cc < nc) {
+        qa[cc] = __ldg(reinterpret_cast<const uint4 *>(qm + qrow) + cc);
+        qb[cc] = __ldg(reinterpret_cast<const uint4 *>(qs + qrow) + cc);
+      }
+    }
+    // scores times the softmax factor, and the row max
+    float mx = -INFINITY;
+    for (int64_t j = l; j < Lk; j += 32) {
+      int d = 0;
+      if (NW != 4) {
+        d = tern_dot<NW>(qa[0], qb[0], sKm[j], sKs[j]);
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          if (cc < nc) d += tern_dot<4>(qa[cc], qb[cc], sKm[j * nc + cc], sKs[j * nc + cc]);
+      }
+      const float x = ((__int2float_rn(d) * sqi) * sk[j]) * c;
+      xw[j] = x;
+      mx = fmaxf(mx, x);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+    float z = 0.0f;
+    for (int64_t j = l; j < Lk; j += 32) {
+      const float e = expf(xw[j] - mx);
+      xw[j] = e;
+      z += e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
+    // keep bits: key j = 32t + l is bit l of mask word t
+    float ksum = 0.0f;
+    int kn = 0;
+    uint32_t *mrow = pm + (bh * Lq + i) * ldp, *srow = ps + (bh * Lq + i) * ldp;
+    for (int64_t t = 0; t * 32 < Lk; ++t) {
+      const int64_t j = t * 32 + l;
+      const float p = j < Lk ? __fdiv_rn(xw[j], z) : 0.0f;
+      const bool keep = p > thr;
+      const uint32_t word = __ballot_sync(FULL, keep);
+      if (keep) ksum += p;
+      kn += keep;
+      if (l == 0) {
+        mrow[t] = word;
+        srow[t] = 0u;
+      }
+    }
+    for (int t = (int)((Lk + 31) / 32) + l; t < ldp; t += 32) {  // padding words
+      mrow[t] = 0u;
+      srow[t] = 0u;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ksum += __shfl_xor_sync(FULL, ksum, o);
+      kn += __shfl_xor_sync(FULL, kn, o);
+    }
+    if (l == 0) pscale[bh * Lq + i] = kn ? __fdiv_rn(ksum, (float)kn) : 0.0f;
+  }
+}
+
+size_t attn_softmax_smem(int64_t Lk, int64_t ld) {
+  const int64_t nc = ld / 4 > 1 ? ld / 4 : 1;
+  return (size_t)Lk * nc * 32 + (size_t)Lk * 4 + (size_t)AS_WARPS * Lk * 4;
+}
+
+template <int NW>
+static cudaError_t launch_softmax_t(const uint32_t *qm, const uint32_t *qs, const float *qscale,
+                                    const uint32_t *km, const uint32_t *ks, const float *kscale,
+                                    int64_t BH, int64_t Lq, int64_t Lk, int64_t ld, float c,
+                                    uint32_t *pm, uint32_t *ps, int64_t ldp, float *pscale,
+                                    cudaStream_t s) {
+  auto kern = k_attn_softmax_pack<NW>;
+  const size_t smem = attn_softmax_smem(Lk, NW == 4 ? ld : 4);
+  static SmemOptIn opt_in;
+  if (cudaError_t e = opt_in(kern, (int)smem)) return e;
+  dim3 grid((unsigned)ceil_div<int64_t>(Lq, AS_ROWS), (unsigned)BH);
+  return launch_pdl(kern, grid, dim3(AS_THREADS), smem, s, qm, qs, qscale, km, ks, kscale, Lq, Lk,
+                    (int)ld, c, pm, ps, (int)ldp, pscale);
+}
+
+cudaError_t launch_attn_softmax(const uint32_t *qm, const uint32_t *qs, const float *qscale,
+                                const uint32_t *km, const uint32_t *ks, const float *kscale,
+                                int64_t BH, int64_t Lq, int64_t Lk, int64_t D, int64_t ld, float c,
+                                uint32_t *pm, uint32_t *ps, int64_t ldp, float *pscale,
+                                cudaStream_t s) {
+  if (BH == 0 || Lq == 0) return cudaSuccess;
+  const int64_t nw = ceil_div<int64_t>(D, 32);
+  if (nw == 1)
+    return launch_softmax_t<1>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, c, pm, ps, ldp, pscale, s);
+  if (nw == 2)
+    return launch_softmax_t<2>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, c, pm, ps, ldp, pscale, s);
+  return launch_softmax_t<4>(qm, qs, qscale, km, ks, kscale, BH, Lq, Lk, ld, c, pm, ps, ldp, pscale, s);
+}
+
 cudaError_t launch_attn_scores(const uint32_t *qm, const uint32_t *qs, const float *qscale,
                                const uint32_t *km, const uint32_t *ks, const float *kscale,
                                int64_t BH, int64_t Lq, int64_t Lk, int64_t D, int64_t ld,

@@ -155,118 +155,189 @@ cudaError_t launch_billm_pack(const float *W, int64_t ldW, int split, const bill
 }
 
 // ================================================================= GEMM
-// CUDA-core path. A warp owns one weight row; lane l owns blocks l, l+32, ...
-// The CTA keeps up to MT activation rows in shared memory as fp32, laid out
-// [m][column-in-block][block] so that the 32 lanes (32 blocks) read 32
-// consecutive words. Per block a lane accumulates, per activation row,
-//   T  = sum over all 128 columns of (+-x)   (b, or b1 at salient columns)
-//   Ts = sum over the sparse group of (+-x)
-//   T1 = sum over salient columns of b1*x,  T2 = the same with b2
-// and adds alpha_c*(T - Ts - T1) + alpha_sp*Ts + alpha1*T1 + alpha2*T2.
-// The sign flip is an XOR of the fp32 sign bit, so +-x costs one LOP3. T is
-// kept as four partial sums (one per 32-column word) so that the adds of a
-// lane form four independent chains. With one activation row the tile is
-// 4*K bytes and several CTAs share an SM.
-constexpr int BG_THREADS = 256, BG_WARPS = BG_THREADS / 32, BG_MT = 4;
-constexpr size_t BG_SMEM_MAX = 160 * 1024;
-template <int MT> constexpr int bg_ctas_per_sm() { return MT == 1 ? 4 : 1; }
+// CUDA-core path, M <= 16 activation rows per pass (larger M with unaligned X
+// loops over groups of 16). Four threads own one weight row (lanes 4r .. 4r+3
+// of a warp; thread p takes the row's 128-column blocks j = p, p + 4, ...), so
+// a warp-load covers 64 contiguous bytes of each of eight rows, and each
+// thread keeps its row's MP output partial sums in registers for all of K.
+// The activations are staged in shared memory as fp32, [block][column][MP]
+// (one 16-byte load gives four rows of one column; blocks 128 * MP + 4 floats
+// apart, so the four threads of a row, on four different blocks, read four
+// different bank groups), a slice of K at a time, with the block sums
+// X_j[m] = sum_c x[m][c] of every 128-column block.
+// Per block of a row (BiLLM "Approach"; the sign plane carries b for
+// non-salient columns and b1 for salient ones):
+//   y += alpha_c * (X_j - 2 * sum_{sign bit 1} x)          every column as +-alpha_c
+//      + sum_{sparse}  (alpha_sp - alpha_c) * b  * x        sparse columns
+//      + sum_{salient} ((alpha1 - alpha_c) * b1 + alpha2 * b2) * x
+// which is the same real value as the pages' four-sum form: one predicated
+// add per weight and row of X, plus a few multiply-adds for the ~10% of
+// columns that are sparse or salient. Partial sums are per 128-column block
+// (fp32 error ~128 * 2^-24 of the block's magnitude), folded into y per block.
+constexpr int BR_THREADS = 256, BR_SPLIT = 4, BR_ROWS = BR_THREADS / BR_SPLIT;
+constexpr size_t BR_SMEM_BUDGET = 160 * 1024;
+constexpr int BR_MAX_NB = 40960 / 128;
 
-template <int MT>
-__global__ void __launch_bounds__(BG_THREADS, bg_ctas_per_sm<MT>())
-k_billm_gemm(const uint16_t *__restrict__ X, int64_t M, int64_t ldX, const uint32_t *__restrict__ sign,
+template <int MP>
+__global__ void __launch_bounds__(BR_THREADS)
+k_billm_rows(const uint16_t *__restrict__ X, int64_t M, int64_t ldX, const uint32_t *__restrict__ sign,
              const uint32_t *__restrict__ gmap, const uint8_t *__restrict__ res,
              const uint8_t *__restrict__ sal, const float *__restrict__ bscale, int64_t N,
-             int64_t K, int64_t ldw, int n_sal, float *__restrict__ Y, int64_t ldY,
+             int64_t K, int64_t ldw, int n_sal, float *__restrict__ Y, int64_t ldY, int slice,
              int32_t *d_status) {
-  extern __shared__ float xs[];  // [MT][128][nb]
+  constexpr int BS = 128 * MP + 4;  // floats per staged block
+  extern __shared__ float4 br_smem4[];
+  float *xs = reinterpret_cast<float *>(br_smem4);     // [slice / 128][BS]
+  float *xsum = xs + (size_t)(slice / 128) * BS;        // [slice / 128][MP]
+  uint8_t *ssal = reinterpret_cast<uint8_t *>(xsum + (slice / 128) * MP);  // [nb][n_sal]
   pdl_trigger();
   pdl_wait();
   const int nb = (int)(K / 128);
-  uint8_t *ssal = reinterpret_cast<uint8_t *>(xs + (size_t)MT * K);
-  for (int i = threadIdx.x; i < nb * n_sal; i += BG_THREADS) ssal[i] = sal[i];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int i = threadIdx.x; i < nb * n_sal; i += BR_THREADS) ssal[i] = sal[i];
+  const int lane = threadIdx.x % 32, part = lane % BR_SPLIT;
+  const int slot = (threadIdx.x / 32) * (32 / BR_SPLIT) + lane / BR_SPLIT;
+  const int64_t groups = ceil_div<int64_t>(N, BR_ROWS);
   bool bad = false;
-  for (int64_t mt0 = 0; mt0 < M; mt0 += MT) {
-    __syncthreads();
-    for (int64_t idx = threadIdx.x; idx < (int64_t)MT * K; idx += BG_THREADS) {
-      const int m = (int)(idx / K);
-      const int64_t k = idx % K;
-      float v = 0.0f;
-      if (mt0 + m < M) {
-        const __half_raw hr = {X[(mt0 + m) * ldX + k]};
-        if ((hr.x & 0x7C00u) == 0x7C00u) bad = true;
-        v = __half2float(__half(hr));
-      }
-      xs[((size_t)m * 128 + (k & 127)) * nb + (k >> 7)] = v;
-    }
-    __syncthreads();
-    for (int64_t n = (int64_t)blockIdx.x * BG_WARPS + warp; n < N; n += (int64_t)gridDim.x * BG_WARPS) {
-      float y[MT];
+
+  for (int64_t mt0 = 0; mt0 < M; mt0 += MP) {
+    for (int64_t rg = blockIdx.x; rg < groups; rg += gridDim.x) {
+      const int64_t n = rg * BR_ROWS + slot;
+      const bool live = n < N;
+      const int64_t nr = live ? n : N - 1;  // rows past N compute a valid row, store nothing
+      float y[MP];
 #pragma unroll
-      for (int m = 0; m < MT; ++m) y[m] = 0.0f;
-      for (int j = lane; j < nb; j += 32) {
-        const uint4 sw = __ldg(reinterpret_cast<const uint4 *>(sign + n * ldw) + j);
-        const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gmap + n * ldw) + j);
-        const float4 sc = __ldg(reinterpret_cast<const float4 *>(bscale) + n * nb + j);
-        const uint32_t rb = res[n * nb + j];
-        float T[MT], Ts[MT], T1[MT], T2[MT], Tq[4][MT];
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          T[m] = Ts[m] = T1[m] = T2[m] = 0.0f;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) Tq[q][m] = 0.0f;
+      for (int m = 0; m < MP; ++m) y[m] = 0.0f;
+      for (int64_t k0 = 0; k0 < K; k0 += slice) {
+        const int cols = (int)(K - k0 < slice ? K - k0 : (int64_t)slice), jb0 = (int)(k0 / 128);
+        // this thread's first block of the slice: its words are requested
+        // before the staging below, which does not need them
+        const int jend = jb0 + cols / 128;
+        int j = jb0 + part;
+        uint4 sw = make_uint4(0, 0, 0, 0), gw = sw;
+        float4 sc = make_float4(0, 0, 0, 0);
+        uint32_t rb = 0;
+        if (j < jend) {
+          sw = __ldg(reinterpret_cast<const uint4 *>(sign + nr * ldw) + j);
+          gw = __ldg(reinterpret_cast<const uint4 *>(gmap + nr * ldw) + j);
+          sc = __ldg(reinterpret_cast<const float4 *>(bscale) + nr * nb + j);
+          rb = res[nr * nb + j];
         }
-        const uint32_t swa[4] = {sw.x, sw.y, sw.z, sw.w}, gwa[4] = {gw.x, gw.y, gw.z, gw.w};
-#pragma unroll 8
-        for (int b = 0; b < 32; ++b) {
+        // stage rows mt0 .. mt0 + MP - 1 of X over this slice (consecutive
+        // threads: consecutive rows of one column, so the stores are
+        // conflict-free and each thread's loads stay in a few L1 sectors),
+        // then the block sums in a fixed order
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < cols * MP; idx += BR_THREADS) {
+          const int m = idx % MP, c = idx / MP;
+          float v = 0.0f;
+          if (mt0 + m < M) {
+            const __half_raw hr = {__ldg(X + (mt0 + m) * ldX + k0 + c)};
+            bad |= (hr.x & 0x7C00u) == 0x7C00u;
+            v = __half2float(__half(hr));
+          }
+          xs[(c >> 7) * BS + (c & 127) * MP + m] = v;
+        }
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < (cols / 128) * MP; idx += BR_THREADS) {
+          const int jl = idx / MP, m = idx % MP;
+          float acc = 0.0f;
+          for (int c = 0; c < 128; ++c) acc += xs[jl * BS + c * MP + m];
+          xsum[jl * MP + m] = acc;
+        }
+        __syncthreads();
+        for (; j < jend; j += BR_SPLIT) {
+          uint4 nsw = make_uint4(0, 0, 0, 0), ngw = nsw;
+          float4 nsc = make_float4(0, 0, 0, 0);
+          uint32_t nrb = 0;
+          if (j + BR_SPLIT < jend) {
+            nsw = __ldg(reinterpret_cast<const uint4 *>(sign + nr * ldw) + j + BR_SPLIT);
+            ngw = __ldg(reinterpret_cast<const uint4 *>(gmap + nr * ldw) + j + BR_SPLIT);
+            nsc = __ldg(reinterpret_cast<const float4 *>(bscale) + nr * nb + j + BR_SPLIT);
+            nrb = res[nr * nb + j + BR_SPLIT];
+          }
+          const float *xj = xs + (size_t)(j - jb0) * BS;
+          const uint32_t swa[4] = {sw.x, sw.y, sw.z, sw.w}, gwa[4] = {gw.x, gw.y, gw.z, gw.w};
+          float neg[MP];
+#pragma unroll
+          for (int m = 0; m < MP; ++m) neg[m] = 0.0f;
+          // sum of x over the columns whose sign bit is 1
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint32_t flip = (swa[q] << (31 - b)) & 0x80000000u;
-            const int c = q * 32 + b;
+            const uint32_t w = swa[q];
+            if (MP == 1) {
 #pragma unroll
-            for (int m = 0; m < MT; ++m)
-              Tq[q][m] += __uint_as_float(__float_as_uint(xs[((size_t)m * 128 + c) * nb + j]) ^ flip);
+              for (int b4 = 0; b4 < 8; ++b4) {
+                const float4 x4 = *reinterpret_cast<const float4 *>(xj + q * 32 + b4 * 4);
+                if (w & (1u << (4 * b4 + 0))) neg[0] += x4.x;
+                if (w & (1u << (4 * b4 + 1))) neg[0] += x4.y;
+                if (w & (1u << (4 * b4 + 2))) neg[0] += x4.z;
+                if (w & (1u << (4 * b4 + 3))) neg[0] += x4.w;
+              }
+            } else {
+#pragma unroll 8
+              for (int b = 0; b < 32; ++b) {
+                if (w & (1u << b)) {
+                  const float *xc = xj + (q * 32 + b) * MP;
+                  if (MP >= 4) {
+#pragma unroll
+                    for (int m4 = 0; m4 < MP; m4 += 4) {
+                      const float4 v = *reinterpret_cast<const float4 *>(xc + m4);
+                      neg[m4] += v.x;
+                      neg[m4 + 1] += v.y;
+                      neg[m4 + 2] += v.z;
+                      neg[m4 + 3] += v.w;
+                    }
+                  } else {
+#pragma unroll
+                    for (int m = 0; m < MP; ++m) neg[m] += xc[m];
+                  }
+                }
+              }
+            }
           }
-        }
+          const float *xsj = xsum + (j - jb0) * MP;
 #pragma unroll
-        for (int m = 0; m < MT; ++m) T[m] = (Tq[0][m] + Tq[1][m]) + (Tq[2][m] + Tq[3][m]);
+          for (int m = 0; m < MP; ++m) y[m] = fmaf(sc.x, fmaf(-2.0f, neg[m], xsj[m]), y[m]);
+          // sparse columns: (alpha_sp - alpha_c) * b * x
+          const float dsp = sc.y - sc.x;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t s = swa[q];
-          uint32_t g = gwa[q];
-          while (g) {
-            const int b = __ffs(g) - 1;
-            g &= g - 1;
-            const uint32_t flip = ((s >> b) & 1u) << 31;
-            const int c = q * 32 + b;
+          for (int q = 0; q < 4; ++q) {
+            uint32_t g = gwa[q];
+            while (g) {
+              const int b = __ffs(g) - 1;
+              g &= g - 1;
+              const float cf = ((swa[q] >> b) & 1u) ? -dsp : dsp;
+              const float *xc = xj + (q * 32 + b) * MP;
 #pragma unroll
-            for (int m = 0; m < MT; ++m)
-              Ts[m] += __uint_as_float(__float_as_uint(xs[((size_t)m * 128 + c) * nb + j]) ^ flip);
+              for (int m = 0; m < MP; ++m) y[m] = fmaf(cf, xc[m], y[m]);
+            }
           }
-        }
-        for (int i = 0; i < n_sal; ++i) {
-          const int c = ssal[j * n_sal + i];
-          const uint32_t f1 = ((swa[c >> 5] >> (c & 31)) & 1u) << 31;
-          const uint32_t f2 = ((rb >> i) & 1u) << 31;
+          // salient columns: (alpha1 - alpha_c) * b1 + alpha2 * b2
+          const float d1 = sc.z - sc.x;
+          for (int i = 0; i < n_sal; ++i) {
+            const int c = ssal[j * n_sal + i];
+            const uint32_t wc = c < 64 ? (c < 32 ? sw.x : sw.y) : (c < 96 ? sw.z : sw.w);
+            const float cf = (((wc >> (c & 31)) & 1u) ? -d1 : d1) +
+                             (((rb >> i) & 1u) ? -sc.w : sc.w);
+            const float *xc = xj + c * MP;
 #pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            const uint32_t xb = __float_as_uint(xs[((size_t)m * 128 + c) * nb + j]);
-            T1[m] += __uint_as_float(xb ^ f1);
-            T2[m] += __uint_as_float(xb ^ f2);
+            for (int m = 0; m < MP; ++m) y[m] = fmaf(cf, xc[m], y[m]);
           }
+          sw = nsw;
+          gw = ngw;
+          sc = nsc;
+          rb = nrb;
         }
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-          y[m] += sc.x * (T[m] - Ts[m] - T1[m]) + sc.y * Ts[m] + sc.z * T1[m] + sc.w * T2[m];
       }
+      // the row's four partial sums (blocks of all four residues)
 #pragma unroll
-      for (int m = 0; m < MT; ++m) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) y[m] += __shfl_xor_sync(FULL, y[m], o);
+      for (int m = 0; m < MP; ++m) {
+        y[m] += __shfl_xor_sync(FULL, y[m], 1);
+        y[m] += __shfl_xor_sync(FULL, y[m], 2);
       }
-      if (lane == 0) {
+      if (live && part == 0) {
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
+        for (int m = 0; m < MP; ++m)
           if (mt0 + m < M) Y[(mt0 + m) * ldY + n] = y[m];
       }
     }
@@ -274,174 +345,36 @@ k_billm_gemm(const uint16_t *__restrict__ X, int64_t M, int64_t ldX, const uint3
   if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
 }
 
-// ------------------------------------------------------------ M = 1 (decode)
-// One activation row: it is staged once per CTA in shared memory as fp32,
-// block-major with a row stride of 132 floats (16-byte aligned, and lanes j
-// reading x[j][c..c+3] hit distinct bank quads), together with the block sums
-// X_j = sum_c x[j][c]. A warp owns a weight row, lane l the blocks l, l+32, ...
-// For a block, sum_c (+-x) = X_j - 2 * sum_{sign bit 1} x: one predicated add
-// per weight, x read four at a time. The sparse group and the salient columns
-// are added as before. The next row's planes and scales are loaded while the
-// current row is summed.
-constexpr int BV_STRIDE = 132;
-
-__global__ void __launch_bounds__(BG_THREADS)
-k_billm_gemv(const uint16_t *__restrict__ X, const uint32_t *__restrict__ sign,
-             const uint32_t *__restrict__ gmap, const uint8_t *__restrict__ res,
-             const uint8_t *__restrict__ sal, const float *__restrict__ bscale, int64_t N,
-             int64_t K, int64_t ldw, int n_sal, float *__restrict__ Y, int32_t *d_status) {
-  extern __shared__ float xs[];  // [nb][BV_STRIDE], then X_j [nb], then salient table
-  pdl_trigger();
-  pdl_wait();
-  const int nb = (int)(K / 128);
-  float *xsum = xs + (size_t)nb * BV_STRIDE;
-  uint8_t *ssal = reinterpret_cast<uint8_t *>(xsum + nb);
-  for (int i = threadIdx.x; i < nb * n_sal; i += BG_THREADS) ssal[i] = sal[i];
-  bool bad = false;
-  for (int64_t k = threadIdx.x; k < K; k += BG_THREADS) {
-    const __half_raw hr = {X[k]};
-    if ((hr.x & 0x7C00u) == 0x7C00u) bad = true;
-    xs[(k >> 7) * BV_STRIDE + (k & 127)] = __half2float(__half(hr));
-  }
-  __syncthreads();
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  for (int j = warp; j < nb; j += BG_WARPS) {  // block sums, fp32, fixed order
-    float v = xs[j * BV_STRIDE + lane] + xs[j * BV_STRIDE + lane + 32] +
-              xs[j * BV_STRIDE + lane + 64] + xs[j * BV_STRIDE + lane + 96];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-    if (lane == 0) xsum[j] = v;
-  }
-  __syncthreads();
-  if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
-
-  const int64_t stride = (int64_t)gridDim.x * BG_WARPS;
-  int64_t n = (int64_t)blockIdx.x * BG_WARPS + warp;
-  // planes and scales of the first block pair of the first row
-  auto load = [&](int64_t row, int j, uint4 &sw, uint4 &gw, float4 &sc, uint32_t &rb) {
-    if (row < N && j < nb) {
-      sw = __ldg(reinterpret_cast<const uint4 *>(sign + row * ldw) + j);
-      gw = __ldg(reinterpret_cast<const uint4 *>(gmap + row * ldw) + j);
-      sc = __ldg(reinterpret_cast<const float4 *>(bscale) + row * nb + j);
-      rb = res[row * nb + j];
-    } else {
-      sw = gw = make_uint4(0, 0, 0, 0);
-      sc = make_float4(0, 0, 0, 0);
-      rb = 0;
-    }
-  };
-  uint4 sw0, gw0, sw1, gw1;
-  float4 sc0, sc1;
-  uint32_t rb0, rb1;
-  load(n, lane, sw0, gw0, sc0, rb0);
-  load(n, lane + 32, sw1, gw1, sc1, rb1);
-  for (; n < N; n += stride) {
-    // next row in flight
-    uint4 nsw0, ngw0, nsw1, ngw1;
-    float4 nsc0, nsc1;
-    uint32_t nrb0, nrb1;
-    load(n + stride, lane, nsw0, ngw0, nsc0, nrb0);
-    load(n + stride, lane + 32, nsw1, ngw1, nsc1, nrb1);
-    float y = 0.0f;
-    for (int jj = 0; jj < nb; jj += 64) {  // this lane's blocks lane + jj, lane + jj + 32
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int j = lane + jj + half * 32;
-        if (j >= nb) continue;
-        uint4 sw = half ? sw1 : sw0, gw = half ? gw1 : gw0;
-        float4 sc = half ? sc1 : sc0;
-        uint32_t rb = half ? rb1 : rb0;
-        if (jj > 0) load(n, j, sw, gw, sc, rb);  // K > 8192: blocks past the first 64
-        const float *xj = xs + j * BV_STRIDE;
-        const uint32_t swa[4] = {sw.x, sw.y, sw.z, sw.w}, gwa[4] = {gw.x, gw.y, gw.z, gw.w};
-        float neg[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-#pragma unroll
-          for (int b4 = 0; b4 < 8; ++b4) {
-            const float4 x4 = *reinterpret_cast<const float4 *>(xj + q * 32 + b4 * 4);
-            const uint32_t s = swa[q] >> (b4 * 4);
-            if (s & 1u) neg[q] += x4.x;
-            if (s & 2u) neg[q] += x4.y;
-            if (s & 4u) neg[q] += x4.z;
-            if (s & 8u) neg[q] += x4.w;
-          }
-        }
-        const float T = xsum[j] - 2.0f * ((neg[0] + neg[1]) + (neg[2] + neg[3]));
-        float Ts = 0.0f, T1 = 0.0f, T2 = 0.0f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t g = gwa[q];
-          while (g) {
-            const int b = __ffs(g) - 1;
-            g &= g - 1;
-            const uint32_t flip = ((swa[q] >> b) & 1u) << 31;
-            Ts += __uint_as_float(__float_as_uint(xj[q * 32 + b]) ^ flip);
-          }
-        }
-        for (int i = 0; i < n_sal; ++i) {
-          const int c = ssal[j * n_sal + i];
-          const uint32_t xb = __float_as_uint(xj[c]);
-          T1 += __uint_as_float(xb ^ (((swa[c >> 5] >> (c & 31)) & 1u) << 31));
-          T2 += __uint_as_float(xb ^ (((rb >> i) & 1u) << 31));
-        }
-        y += sc.x * (T - Ts - T1) + sc.y * Ts + sc.z * T1 + sc.w * T2;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(FULL, y, o);
-    if (lane == 0) Y[n] = y;
-    sw0 = nsw0; gw0 = ngw0; sc0 = nsc0; rb0 = nrb0;
-    sw1 = nsw1; gw1 = ngw1; sc1 = nsc1; rb1 = nrb1;
-  }
+// Columns of K staged per pass: all of K when it fits, else a multiple of 512
+// (every thread then has blocks in each slice).
+static int br_slice(int mp, int64_t K) {
+  // per 128 columns: the staged block (128 * mp + 4 floats) and its mp sums
+  const int64_t per_block = ((int64_t)128 * mp + 4 + mp) * 4;
+  const int64_t fit = (int64_t)(BR_SMEM_BUDGET - BR_MAX_NB * 8) / per_block * 128;
+  if (fit >= K) return (int)K;
+  return (int)std::max<int64_t>(512, fit / 512 * 512);
 }
 
-static cudaError_t launch_billm_gemv(const uint16_t *X, const billm_weights *W, float *Y,
-                                     int32_t *d_status, cudaStream_t s) {
-  const size_t smem = (size_t)(W->K / 128) * (BV_STRIDE + 1) * 4 + 8 * (W->K / 128);
-  static cudaError_t attr = cudaFuncSetAttribute(
-      k_billm_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BG_SMEM_MAX);
-  if (attr != cudaSuccess) return attr;
+template <int MP>
+static cudaError_t launch_br_t(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,
+                               float *Y, int64_t ldY, int32_t *d_status, cudaStream_t s) {
+  auto kern = k_billm_rows<MP>;
+  const int slice = br_slice(MP, W->K);
+  const size_t smem = (size_t)(slice / 128) * (128 * MP + 4 + MP) * 4 +
+                      (size_t)(W->K / 128) * W->n_sal;
+  static SmemOptIn opt_in;
+  if (cudaError_t e = opt_in(kern, (int)smem)) return e;
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_billm_gemv, BG_THREADS, smem) !=
-          cudaSuccess || per_sm < 1)
-    per_sm = 1;
-  const int64_t blocks =
-      std::min<int64_t>(ceil_div<int64_t>(W->N, BG_WARPS), (int64_t)sms * per_sm);
-  return launch_pdl(k_billm_gemv, dim3((unsigned)blocks), dim3(BG_THREADS), smem, s, X, W->sign,
-                    W->gmap, W->res, W->sal, W->bscale, W->N, W->K, W->ldw_words, (int)W->n_sal,
-                    Y, d_status);
-}
-
-int billm_gemm_mt(int64_t K) {
-  const int64_t per = K * 4;
-  int mt = BG_MT;
-  while (mt > 1 && (size_t)(mt * per) + 8 * (K / 128) > BG_SMEM_MAX) mt /= 2;
-  return ((size_t)(mt * per) + 8 * (K / 128) > BG_SMEM_MAX) ? 0 : mt;
-}
-
-template <int MT>
-static cudaError_t launch_bg_t(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,
-                               float *Y, int64_t ldY, int32_t *d_status, cudaStream_t s) {
-  auto kern = k_billm_gemm<MT>;
-  static cudaError_t attr =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BG_SMEM_MAX);
-  if (attr != cudaSuccess) return attr;
-  const size_t smem = (size_t)MT * W->K * 4 + 8 * (W->K / 128);
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int per_sm = 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, BG_THREADS, smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, BR_THREADS, smem) != cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
   const int64_t blocks =
-      std::min<int64_t>(ceil_div<int64_t>(W->N, BG_WARPS), (int64_t)sms * per_sm);
-  return launch_pdl(kern, dim3((unsigned)blocks), dim3(BG_THREADS), smem, s, X, M, ldX, W->sign,
+      std::min<int64_t>(ceil_div<int64_t>(W->N, BR_ROWS), (int64_t)sms * per_sm);
+  return launch_pdl(kern, dim3((unsigned)blocks), dim3(BR_THREADS), smem, s, X, M, ldX, W->sign,
                     W->gmap, W->res, W->sal, W->bscale, W->N, W->K, W->ldw_words, (int)W->n_sal, Y,
-                    ldY, d_status);
+                    ldY, slice, d_status);
 }
 
 cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,
@@ -451,12 +384,11 @@ cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const b
     const cudaError_t e = launch_billm_gemm_tc(X, M, ldX, W, Y, ldY, d_status, s);
     if (e != cudaErrorNotSupported) return e;
   }
-  if (M == 1 && (size_t)(W->K / 128) * (BV_STRIDE + 1) * 4 + 8 * (W->K / 128) <= BG_SMEM_MAX)
-    return launch_billm_gemv(X, W, Y, d_status, s);
-  const int mt = billm_gemm_mt(W->K);
-  if (mt >= 4 && M >= 4) return launch_bg_t<4>(X, M, ldX, W, Y, ldY, d_status, s);
-  if (mt >= 2 && M >= 2) return launch_bg_t<2>(X, M, ldX, W, Y, ldY, d_status, s);
-  return launch_bg_t<1>(X, M, ldX, W, Y, ldY, d_status, s);
+  if (M == 1) return launch_br_t<1>(X, M, ldX, W, Y, ldY, d_status, s);
+  if (M == 2) return launch_br_t<2>(X, M, ldX, W, Y, ldY, d_status, s);
+  if (M <= 4) return launch_br_t<4>(X, M, ldX, W, Y, ldY, d_status, s);
+  if (M <= 8) return launch_br_t<8>(X, M, ldX, W, Y, ldY, d_status, s);
+  return launch_br_t<16>(X, M, ldX, W, Y, ldY, d_status, s);
 }
 
 }  // namespace bwta

@@ -68,6 +68,7 @@ struct BtSync {
   uint64_t drain;
   uint32_t tmem_base;
   int32_t timeout;
+  int32_t undrained;  // a post-timeout drain ran out of time
 };
 
 template <int BN>
@@ -141,6 +142,7 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
     }
     mbar_init(&sy->drain, 1);
     sy->timeout = 0;
+    sy->undrained = 0;
     mbar_fence_init();
   }
   if (warp == BT_ISSUER) {
@@ -178,8 +180,10 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
           tma_load_2d(stages + s * Sh::STAGE, &map_x, kb * BT_KB, m0, &sy->xfull[s]);
         }
       }
+      // a stage is reloaded only after the MMAs that read it, which waited for
+      // its load: the last S loads are the only ones that can be pending
       for (uint32_t j = g > (uint32_t)S ? g - S : 0; j < g; ++j)
-        mbar_wait(&sy->xfull[j % S], (j / S) & 1, 100000000ull);
+        if (!mbar_wait(&sy->xfull[j % S], (j / S) & 1, DRAIN_NS)) sy->undrained = 1;
     }
     __syncwarp();
   } else if (warp == BT_ISSUER) {
@@ -212,7 +216,7 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
         }
       }
       tc_commit(&sy->drain);
-      mbar_wait(&sy->drain, 0, 100000000ull);
+      if (!mbar_wait(&sy->drain, 0, DRAIN_NS)) sy->undrained = 1;
     }
     __syncwarp();
   } else if (warp < BT_EXPAND) {
@@ -355,16 +359,18 @@ k_billm_gemm_tc(const __grid_constant__ CUtensorMap map_x, const uint32_t *__res
     tc_fence_after();
     tmem_dealloc(tmem, Sh::TMEM_COLS);
   }
-  if (threadIdx.x == 0 && sy->timeout) flag_status(d_status, BWTA_STATUS_TIMEOUT);
+  // TMEM is released even after a drain ran out of time (a later CTA on this
+  // SM would otherwise block in its allocation); the DRAIN flag reports it
+  if (threadIdx.x == 0 && sy->timeout)
+    flag_status(d_status, BWTA_STATUS_TIMEOUT | (sy->undrained ? BWTA_STATUS_DRAIN : 0));
 }
 
 template <int BN>
 static cudaError_t launch_bt_t(const CUtensorMap &mx, const billm_weights *W, int64_t M, float *Y,
                                int64_t ldY, int32_t *d_status, cudaStream_t s) {
   auto kern = k_billm_gemm_tc<BN>;
-  static cudaError_t attr =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bt_smem<BN>());
-  if (attr != cudaSuccess) return attr;
+  static SmemOptIn opt_in;
+  if (cudaError_t e = opt_in(kern, (int)bt_smem<BN>())) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

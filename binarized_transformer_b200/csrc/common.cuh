@@ -5,11 +5,43 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#ifndef __CUDACC_RTC__
+#include <atomic>
+#endif
+
 #include "../../include/bwta.h"
 
 namespace bwta {
 
 constexpr unsigned FULL = 0xffffffffu;
+
+// Bound of the waits that let a CTA's own copies and MMAs finish after one of
+// its barrier waits timed out (the normal waits are bounded at 2 s).
+constexpr uint64_t DRAIN_NS = 1000000000ull;
+
+#ifndef __CUDACC_RTC__
+// The >48 KB dynamic shared-memory opt-in of one kernel, made once per device
+// (the device current at the call). Only a success is remembered, so a call
+// that failed is retried on the next launch.
+class SmemOptIn {
+ public:
+  template <typename Kern>
+  cudaError_t operator()(Kern *kern, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cached = dev >= 0 && dev < kDevices;
+    if (cached && set_[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && cached) set_[dev].store(bytes, std::memory_order_release);
+    return e;
+  }
+
+ private:
+  static constexpr int kDevices = 64;
+  std::atomic<int> set_[kDevices] = {};
+};
+#endif
 
 // ----------------------------------------------------------------- status
 __device__ __forceinline__ void flag_status(int32_t *d_status, int32_t flag) {
@@ -128,21 +160,40 @@ cudaError_t launch_gemm_tiled(const uint32_t *am, const uint32_t *as, const floa
                               int64_t M, int64_t lda, const uint32_t *wb, const float *wscale,
                               int64_t N, int64_t ldw, int64_t K, int64_t group, float *Y,
                               int64_t ldY, int32_t *dots, int64_t ldD, int32_t *d_status,
-                              cudaStream_t s);
-cudaError_t launch_gemv(const uint32_t *am, const uint32_t *as, const float *ascale, int64_t M,
-                        int64_t lda, const uint32_t *wb, const float *wscale, int64_t N,
-                        int64_t ldw, int64_t K, int64_t group, float *Y, int64_t ldY,
-                        int32_t *dots, int64_t ldD, bool weights_ready, cudaStream_t s);
-bool gemv_fits(int64_t M, int64_t lda, int64_t K, int64_t group);
-bool linear_decode_fits(int64_t M, int64_t K);
-cudaError_t launch_linear_decode(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int mode,
-                                 const uint32_t *wb, const float *wscale, int64_t N, int64_t ldw,
-                                 int64_t group, float *Y, int64_t ldY, int32_t *dots, int64_t ldD,
-                                 bool ready, int32_t *d_status, cudaStream_t s);
+                              uint64_t stall_ns, cudaStream_t s);
+// One decode projection (M <= 8 activation rows): fp16 rows X to ternarize in
+// the kernel (fused) or packed planes am / as / ascale.
+struct DecodeSpec {
+  const uint16_t *X;
+  int64_t ldX;
+  const uint32_t *am, *as;
+  const float *ascale;
+  int64_t lda;
+  int64_t M, K;
+  const uint32_t *wbits;
+  const float *wscale;
+  int64_t N, ldw, group;
+  float *Y;
+  int64_t ldY;
+  int32_t *dots;
+  int64_t ldD;
+};
+bool decode_fits(int64_t M, int64_t K);
+int decode_max_jobs();
+size_t decode_act_bytes(int64_t M, int64_t K);
+size_t decode_max_act_bytes();
+cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mode, bool ready,
+                          int32_t *d_status, cudaStream_t s);
 cudaError_t launch_attn_scores(const uint32_t *qm, const uint32_t *qs, const float *qscale,
                                const uint32_t *km, const uint32_t *ks, const float *kscale,
                                int64_t BH, int64_t Lq, int64_t Lk, int64_t D, int64_t ld,
                                int32_t *Si, float *Sf, cudaStream_t s);
+size_t attn_softmax_smem(int64_t Lk, int64_t ld);
+cudaError_t launch_attn_softmax(const uint32_t *qm, const uint32_t *qs, const float *qscale,
+                                const uint32_t *km, const uint32_t *ks, const float *kscale,
+                                int64_t BH, int64_t Lq, int64_t Lk, int64_t D, int64_t ld, float c,
+                                uint32_t *pm, uint32_t *ps, int64_t ldp, float *pscale,
+                                cudaStream_t s);
 cudaError_t launch_billm_pack(const float *W, int64_t ldW, int split, const billm_weights *out,
                               int32_t *d_status, cudaStream_t s);
 cudaError_t launch_billm_gemm_tc(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,

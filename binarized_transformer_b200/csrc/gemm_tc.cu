@@ -79,6 +79,7 @@ struct TcBarriers {
   uint64_t drain;             // all MMAs of the CTA complete (teardown)
   uint32_t tmem_base;
   int32_t timeout;
+  int32_t undrained;          // a post-timeout drain ran out of time
 };
 
 // Bounded wait that also records a timeout for the whole CTA.
@@ -155,6 +156,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
     }
     mbar_init(&bars->drain, 1);
     bars->timeout = 0;
+    bars->undrained = 0;
     mbar_fence_init();
   }
   if (warp == TC_ISSUER) {
@@ -188,9 +190,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
         }
       }
       // Loads still in flight (after a timeout) land before the CTA exits; in
-      // a normal run these phases are complete already.
+      // a normal run these phases are complete already. A stage is reloaded
+      // only after the MMAs that read its previous load, which waited for that
+      // load, so the last TC_STAGES loads are the only ones that can be pending.
       for (uint32_t j = g > TC_STAGES ? g - TC_STAGES : 0; j < g; ++j)
-        mbar_wait(&bars->full[j % TC_STAGES], (j / TC_STAGES) & 1, 100000000ull);
+        if (!mbar_wait(&bars->full[j % TC_STAGES], (j / TC_STAGES) & 1, DRAIN_NS))
+          bars->undrained = 1;
     }
     __syncwarp();
   } else if (warp == TC_ISSUER) {
@@ -234,7 +239,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
       }
       // Every MMA issued has completed before TMEM is released.
       tc_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0, 100000000ull);
+      if (!mbar_wait(&bars->drain, 0, DRAIN_NS)) bars->undrained = 1;
     }
     __syncwarp();
   } else if (warp < 4) {
@@ -334,13 +339,17 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
     }
   }
 
+  // TMEM is released even when a drain ran out of time: a later CTA on this SM
+  // would otherwise block in its allocation for good. The DRAIN flag tells the
+  // caller that the context is no longer to be trusted.
   tc_fence_before();
   __syncthreads();
   if (warp == TC_ISSUER) {
     tc_fence_after();
     tmem_dealloc(tmem, TC_TMEM_COLS);
   }
-  if (threadIdx.x == 0 && bars->timeout) flag_status(d_status, BWTA_STATUS_TIMEOUT);
+  if (threadIdx.x == 0 && bars->timeout)
+    flag_status(d_status, BWTA_STATUS_TIMEOUT | (bars->undrained ? BWTA_STATUS_DRAIN : 0));
 }
 
 template <bool GROUPED, bool WANT_Y, bool WANT_DOTS>
@@ -349,9 +358,8 @@ static cudaError_t launch_tc_t(const CUtensorMap &mx, const CUtensorMap &mw, con
                                int64_t G, float *Y, int64_t ldY, int32_t *dots, int64_t ldD,
                                int32_t *d_status, cudaStream_t s) {
   auto kern = k_gemm_tc<GROUPED, WANT_Y, WANT_DOTS>;
-  static cudaError_t attr =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM);
-  if (attr != cudaSuccess) return attr;
+  static SmemOptIn opt_in;
+  if (cudaError_t e = opt_in(kern, (int)TC_SMEM)) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

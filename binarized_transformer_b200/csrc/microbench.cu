@@ -6,6 +6,8 @@
 //  * legacy warp-level MMA rates: b1 AND+POPC (m16n8k256), s8 (m16n8k32) and
 //    f16 (m16n8k16), for comparison with the CUDA-core path;
 //  * HBM streaming read and write bandwidth.
+//  * the bit GEMM's inner mix per 4-word chunk (4 LOP3 m & (a ^ w), a
+//    carry-save adder of 2 LOP3s, 3 POPCs, adds): the ceiling of that kernel;
 // Each kernel keeps independent dependency chains per thread so that issue
 // throughput, not latency, bounds it; results feed a sink so nothing is
 // optimized away. The caller times the launches with CUDA events.
@@ -38,6 +40,38 @@ __global__ void mb_wordop(uint32_t *sink, int iters, uint32_t seed) {
   uint32_t r = 0;
 #pragma unroll
   for (int i = 0; i < CH; ++i) r ^= acc[i];
+  if (r == 0x12345678u) sink[0] = r;
+}
+
+// The bit GEMM's own inner mix for one output and one 4-word chunk: four
+// m & (a ^ w) LOP3s, a carry-save full adder over three of them (two LOP3s),
+// three POPCs and the adds that weight them, acc += popc(s) + popc(t3) +
+// 2 * popc(c). The accumulator stands in for the weight words so that every
+// iteration depends on the last; 4 word-ops per chain and iteration.
+__global__ void mb_popc4(uint32_t *sink, int iters, uint32_t seed) {
+  constexpr int C4 = 8;
+  uint32_t m[4], a[4], acc[C4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m[i] = seed ^ (0x85EBCA6Bu * (i + 1) + threadIdx.x);
+    a[i] = seed * 0x9E3779B9u + 0x27D4EB2Fu * i + threadIdx.x;
+  }
+#pragma unroll
+  for (int c = 0; c < C4; ++c) acc[c] = c * 0x61C88647u;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int c = 0; c < C4; ++c) {
+      const uint32_t t0 = lop3_and_xor(m[0], a[0], acc[c]), t1 = lop3_and_xor(m[1], a[1], acc[c]);
+      const uint32_t t2 = lop3_and_xor(m[2], a[2], acc[c]), t3 = lop3_and_xor(m[3], a[3], acc[c]);
+      uint32_t s, cy;
+      asm volatile("lop3.b32 %0, %1, %2, %3, 0x96;" : "=r"(s) : "r"(t0), "r"(t1), "r"(t2));
+      asm volatile("lop3.b32 %0, %1, %2, %3, 0xE8;" : "=r"(cy) : "r"(t0), "r"(t1), "r"(t2));
+      acc[c] += __popc(s) + __popc(t3) + 2 * __popc(cy);
+    }
+  }
+  uint32_t r = 0;
+#pragma unroll
+  for (int c = 0; c < C4; ++c) r ^= acc[c];
   if (r == 0x12345678u) sink[0] = r;
 }
 
@@ -208,7 +242,7 @@ __global__ void mb_write(uint4 *__restrict__ p, size_t n, uint32_t v) {
 extern "C" {
 
 // Ops counted per thread per iteration (the caller multiplies by threads*iters):
-//   wordop/lop3/popc/imad: 16; mma_*: 4 instructions per thread-iteration,
+//   wordop/lop3/popc/imad: 16; popc4: 32 word-ops; mma_*: 4 instructions per thread-iteration,
 //   i.e. 4/32 per thread of the warp-wide instruction.
 int bwta_mb_launch(int kind, int blocks, int threads, int iters, uint32_t *sink, void *stream) {
   cudaStream_t s = (cudaStream_t)stream;
@@ -220,6 +254,7 @@ int bwta_mb_launch(int kind, int blocks, int threads, int iters, uint32_t *sink,
     case 4: mb_mma_b1<<<blocks, threads, 0, s>>>(sink, iters, 1u); break;
     case 5: mb_mma_s8<<<blocks, threads, 0, s>>>(sink, iters, 1u); break;
     case 6: mb_mma_f16<<<blocks, threads, 0, s>>>(sink, iters, 1u); break;
+    case 7: mb_popc4<<<blocks, threads, 0, s>>>(sink, iters, 1u); break;
     default: return -1;
   }
   return (int)cudaGetLastError();

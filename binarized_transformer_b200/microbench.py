@@ -1,7 +1,10 @@
 """Measured ceilings for the roofline of each kernel (libbwta_microbench.so).
 
-* word-op rate: acc += popc(m & (a ^ w)) -- one LOP3, one POPC, one add, the
-  inner loop of the bit GEMM; one word-op is 32 multiply-adds = 64 binary ops.
+* word-op rate: acc += popc(m & (a ^ w)) -- one LOP3, one POPC, one add; one
+  word-op is 32 multiply-adds = 64 binary ops.
+* popc4 rate: the bit GEMM's own inner mix per 4-word chunk (four LOP3s, a
+  carry-save adder of two LOP3s, three POPCs, the adds), in word-ops: the
+  ceiling the tiled GEMM is measured against.
 * LOP3, POPC(+add), IMAD issue rates on their own.
 * legacy warp MMA rates: b1 AND+POPC (bit products), s8, f16 (fp32 accumulate).
 * HBM streaming read and write bandwidth over a 1 GiB buffer.
@@ -17,9 +20,10 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
 
-KINDS = {"wordop": 0, "lop3": 1, "popc": 2, "imad": 3, "mma_b1": 4, "mma_s8": 5, "mma_f16": 6}
+KINDS = {"wordop": 0, "lop3": 1, "popc": 2, "imad": 3, "mma_b1": 4, "mma_s8": 5, "mma_f16": 6,
+         "popc4": 7}
 # work per thread per loop iteration
-_PER_THREAD_ITER = {"wordop": 16, "lop3": 16, "popc": 16, "imad": 16}
+_PER_THREAD_ITER = {"wordop": 16, "lop3": 16, "popc": 16, "imad": 16, "popc4": 32}
 _MMA_WORK = {"mma_b1": 16 * 8 * 256, "mma_s8": 16 * 8 * 32, "mma_f16": 16 * 8 * 16}  # MACs / instr
 
 

@@ -63,6 +63,12 @@ typedef enum bwta_status {
 /* device-side status flags, OR-ed into *d_status */
 #define BWTA_STATUS_NONFINITE 0x1 /* an input held Inf or NaN; outputs of that row are unspecified */
 #define BWTA_STATUS_TIMEOUT 0x2   /* a bounded wait inside a kernel gave up; outputs are unspecified */
+/* After a timeout a kernel lets its own copies and tensor-core operations in
+ * flight finish (bounded at 1 s) before it releases tensor memory and exits.
+ * This flag says that bound ran out as well: the kernel exited anyway, so work
+ * of that launch may still have been running. Treat the CUDA context as
+ * unreliable and reset it. */
+#define BWTA_STATUS_DRAIN 0x4
 
 #define BWTA_TERNARY 0
 #define BWTA_BINARY 1
@@ -140,9 +146,8 @@ int bwta_gemm_tc(const uint8_t *a_e4m3, int64_t ld_e4m3, const float *a_scale, i
  *     Y[m][n] = fp32: acc = 0; for g ascending: acc = fma((float)d_g, alpha[n][g], acc);
  *               Y = acc * a_scale[m]
  *     dots[m][n] = sum_g d_g  (exact int32)
- * M <= 8 runs the decode GEMV kernel (its fp32 sum over groups is a tree, not
- * the serial order above; its dots are the same integers), larger M the tiled
- * GEMM, which follows the serial order exactly.
+ * M <= 8 (and K <= 16384) runs the decode GEMV kernel, larger M the tiled
+ * GEMM; both follow the serial order above, so Y is the same bit for bit.
  *  a_mask, a_sign  uint32 [M][lda_words]; a_scale fp32 [M]
  *  wbits           uint32 [N][ldw_words]; wscale fp32 [N][G]
  *  Y               fp32 [M][ldY] out, may be NULL
@@ -176,8 +181,7 @@ int bwta_gemm_ex(const uint32_t *a_mask, const uint32_t *a_sign, const float *a_
  * and multiply them by packed binary weights, without writing the activation
  * planes to memory (BWTA abstract: ternary activations; bit-packed MatMul).
  * Equivalent to bwta_quantize_pack_acts followed by bwta_gemm: the same planes
- * and scales bit for bit, the same integer dots; fp32 outputs within the
- * tolerance of the decode GEMV (group terms summed as a tree).
+ * and scales, the same integer dots and the same fp32 outputs, bit for bit.
  *  X          fp16 bits [M][ldX], any alignment
  *  mode, thresh_ratio   as bwta_quantize_pack_acts
  *  wbits, wscale, N, ldw_words, group, Y, ldY, dots, ldD   as bwta_gemm
@@ -188,6 +192,37 @@ int bwta_linear_decode(const uint16_t *X, int64_t M, int64_t K, int64_t ldX, int
                        float thresh_ratio, const uint32_t *wbits, const float *wscale, int64_t N,
                        int64_t ldw_words, int64_t group, float *Y, int64_t ldY, int32_t *dots,
                        int64_t ldD, uint32_t flags, int32_t *d_status, bwta_stream_t stream);
+
+/* One projection of a batched decode call: the arguments of bwta_linear_decode. */
+typedef struct bwta_decode_job {
+  const uint16_t *X; /* fp16 bits [M][ldX] */
+  int64_t M, K, ldX;
+  const uint32_t *wbits; /* [N][ldw_words] */
+  const float *wscale;   /* [N][G] */
+  int64_t N, ldw_words, group;
+  float *Y; /* [M][ldY], may be NULL */
+  int64_t ldY;
+  int32_t *dots; /* [M][ldD], may be NULL (not both) */
+  int64_t ldD;
+} bwta_decode_job;
+
+/* Several independent decode projections in ONE launch (BWTA abstract: the
+ * bit-packed MatMul, here at decode, where each product streams its weights
+ * once and a launch per projection would cost more than the stream itself):
+ * e.g. the q/k/v or gate/up projections of one layer, or projections of
+ * different layers that do not depend on one another. Every job is computed
+ * exactly as bwta_linear_decode computes it alone (same planes, dots and fp32
+ * outputs, bit for bit); the jobs must not write overlapping outputs.
+ *  jobs       host array of njobs descriptors (read during the call only)
+ *  njobs      0 .. 8
+ *  mode, thresh_ratio, flags   as bwta_linear_decode, for every job
+ *  Limits: per job as bwta_linear_decode; the packed activations of all jobs
+ *  (36 bytes per 128 elements per row, rounded to 16 bytes per job) must fit in
+ *  48 KB of shared memory; else UNSUPPORTED.
+ *  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; NONFINITE flag. */
+int bwta_linear_decode_batched(const bwta_decode_job *jobs, int64_t njobs, int mode,
+                               float thresh_ratio, uint32_t flags, int32_t *d_status,
+                               bwta_stream_t stream);
 
 /* Ternary attention scores Q . K^T per batch*head (BWTA abstract: binary /
  * ternary MatMul for the attention operators). Both operands come from
@@ -251,6 +286,25 @@ int billm_pack_weights(const float *W, int64_t ldW, int split, const billm_weigh
  *  TIMEOUT flags. */
 int billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W, float *Y,
                int64_t ldY, int32_t *d_status, bwta_stream_t stream);
+
+/* Failure-path self-test of the bounded waits. The paper has no counterpart:
+ * this exercises the library's own error handling. It runs the tiled kernel of
+ * bwta_gemm (arguments as there; M must be > 8) with one extra wait per CTA, on
+ * a shared-memory barrier that nothing ever completes, bounded by
+ * wait_limit_ns. Every CTA then takes the kernel's timeout path: it ORs
+ * BWTA_STATUS_TIMEOUT into *d_status, lets the tile loads it issued land, and
+ * returns. Y and dots are left unspecified. No fault is raised and the context
+ * stays usable: later calls compute normally.
+ *  wait_limit_ns  1 .. 2000000000
+ *  d_status       required (device int32)
+ *  Errors: as bwta_gemm; INVALID_ARG if M <= 8, d_status is NULL or the limit
+ *  is out of range. */
+int bwta_selftest_gemm_timeout(const uint32_t *a_mask, const uint32_t *a_sign,
+                               const float *a_scale, int64_t M, int64_t lda_words,
+                               const uint32_t *wbits, const float *wscale, int64_t N,
+                               int64_t ldw_words, int64_t K, int64_t group, float *Y, int64_t ldY,
+                               int32_t *dots, int64_t ldD, int64_t wait_limit_ns,
+                               int32_t *d_status, bwta_stream_t stream);
 
 /* Library version string, e.g. "bwta 0.1 sm_100a". */
 const char *bwta_version(void);

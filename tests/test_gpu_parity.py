@@ -171,7 +171,9 @@ def test_gemm_tiled_small(M, N, K, group):
 def test_gemv_small(M, N, K, group):
     X = workloads.edge_acts(M, K, "student", tag=M)
     W = workloads.edge_weights(N, K, tag=M)
-    run_linear(X, W, group)
+    Y, yrep = run_linear(X, W, group)
+    # the decode GEMV folds the groups in the oracle's serial fp32 order
+    np.testing.assert_array_equal(Y.view(np.uint32), yrep.view(np.uint32))
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (1, 300, 11008), (3, 1000, 4096)])
@@ -190,6 +192,7 @@ def test_gemv_weights_ready_flag(M, N, K):
         torch.cuda.synchronize()
         np.testing.assert_array_equal(D.cpu().numpy(), ref["dots"])
         assert_close_rel(Y.cpu().numpy(), ref["yref"], ref["mag"], what="gemv ready")
+        np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint32), ref["yrep"].view(np.uint32))
 
 
 @pytest.mark.parametrize("ready", [False, True])
@@ -215,6 +218,7 @@ def test_linear_decode_fused(M, N, K, group, ready):
     dcheck()
     np.testing.assert_array_equal(Dv.cpu().numpy(), ref["dots"])
     assert_close_rel(Yv.cpu().numpy(), ref["yref"], ref["mag"] if group else None, what="decode")
+    np.testing.assert_array_equal(Yv.cpu().numpy().view(np.uint32), ref["yrep"].view(np.uint32))
 
 
 def test_linear_decode_binary_and_zero_rows():
