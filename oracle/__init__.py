@@ -210,7 +210,7 @@ def billm_quantize_rows(W, sal, n0, n1, block=128, split=True):
     b1 = np.zeros((R, K), np.int8)
     b2 = np.zeros((R, K), np.int8)
     scales = np.zeros((R, K // block, 4), np.float32)
-    _check(lib().orc_billm_quantize_rows(_p(W), n0, n1, K, K, block, n_sal, int(bool(split)),
+    _check(lib().orc_billm_quantize_rows(_p(W), n0, n1, K, K, block, n_sal, int(split),
                                          _p(sal), _p(cat), _p(b1), _p(b2), _p(scales)),
            "billm_quantize_rows")
     return dict(cat=cat, b1=b1, b2=b2, scales=scales, sal=sal, block=block)

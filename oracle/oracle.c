@@ -35,6 +35,13 @@
  *  R5  BiLLM break-point: p = 0.5 * max|w| over the non-salient weights of
  *      one row inside one block; sparse group = {|w| > p}.
  *  R6  BiLLM scales are rounded to fp32 before any further use.
+ *  R17 attention probabilities are ternarized like activations: kept iff
+ *      p > 0.5 * mean(p) = 1/(2L) (a softmax row has mean 1/L); scale = mean
+ *      of the kept p.
+ *  R18 BiLLM's "optimal splitting search": the break-point is the non-salient
+ *      magnitude of the row-block that minimizes the squared binarization
+ *      error of the two groups (each scaled by its mean magnitude); ties go to
+ *      the smaller break-point.
  *
  * Arithmetic of the fp16 magnitudes: every finite fp16 value is an integer
  * multiple of 2^-24, so |x| * 2^24 is an exact integer below 2^40 and sums of
@@ -343,14 +350,49 @@ int orc_billm_salient(const float *W, int64_t N, int64_t K, int64_t ldW, int64_t
   return ORC_OK;
 }
 
+/* The squared binarization error of the non-salient weights of one
+ * row-block when split at break-point p ([BiLLM] "Approach": the bell-shaped
+ * non-salient weights are split at a break-point into a concentrated and a
+ * sparse group, each binarized with its own scale). With a group's scale the
+ * mean of its magnitudes (the L2-optimal scale of a sign-binarized group) and
+ * (w - a*sign(w))^2 = (|w| - a)^2:
+ *   E(p) = sum_{|w| <= p} (|w| - a_c)^2 + sum_{|w| > p} (|w| - a_s)^2
+ * Every sum in fp64, columns ascending; an empty group contributes 0. */
+static double split_error(const float *w, const int8_t *cat, int64_t block, double p) {
+  double sc = 0.0, ss = 0.0;
+  int64_t nc = 0, ns = 0;
+  for (int64_t c = 0; c < block; ++c) {
+    if (cat[c] == 2) continue;
+    const double aw = fabs((double)w[c]);
+    if (aw <= p) {
+      sc += aw;
+      ++nc;
+    } else {
+      ss += aw;
+      ++ns;
+    }
+  }
+  const double ac = nc ? sc / (double)nc : 0.0, as = ns ? ss / (double)ns : 0.0;
+  double e = 0.0;
+  for (int64_t c = 0; c < block; ++c) {
+    if (cat[c] == 2) continue;
+    const double aw = fabs((double)w[c]);
+    const double d = aw - (aw <= p ? ac : as);
+    e += d * d;
+  }
+  return e;
+}
+
 /* Per-row BiLLM binarization of rows [n0, n1) ([BiLLM] Approach; R5, R6).
  * Inside block j of row n:
  *   salient columns:  alpha1 = mean|w|, b1 = sign(w);
  *                     r = w - alpha1*b1, alpha2 = mean|r|, b2 = sign(r)
  *                     (residual binarization: w ~ alpha1*b1 + alpha2*b2);
- *   other columns:    p = 0.5 * max|w|; sparse group = {|w| > p} (only when
- *                     split != 0), concentrated = the rest; each group:
- *                     alpha = mean|w| over its members (0 if empty), b = sign(w).
+ *   other columns:    split == 1: p = 0.5 * max|w| (R5); split == 2: p is the
+ *                     searched break-point (R18, split_error above);
+ *                     sparse group = {|w| > p} (none when split == 0),
+ *                     concentrated = the rest; each group: alpha = mean|w|
+ *                     over its members (0 if empty), b = sign(w).
  * Outputs for row r = n - n0:
  *   cat[r*K + k]   0 concentrated, 1 sparse, 2 salient
  *   b1[r*K + k]    +-1 (b for non-salient, b1 for salient)
@@ -403,13 +445,30 @@ int orc_billm_quantize_rows(const float *W, int64_t n0, int64_t n1, int64_t K, i
           double aw = fabs((double)row[base + c]);
           if (aw > maxabs) maxabs = aw;
         }
+      /* split == 2: the searched break-point (reading R18). Candidates are the
+       * block's non-salient magnitudes; the chosen p minimizes the squared
+       * binarization error of the two groups; ties go to the smaller p. */
+      double pbest = maxabs;
+      if (split == 2) {
+        double ebest = INFINITY;
+        for (int64_t c0 = 0; c0 < block; ++c0) {
+          if (cat[r * K + base + c0] == 2) continue;
+          const double p = fabs((double)row[base + c0]);
+          const double e = split_error(row + base, cat + r * K + base, block, p);
+          if (e < ebest || (e == ebest && p < pbest)) {
+            ebest = e;
+            pbest = p;
+          }
+        }
+      }
       double sum_c = 0.0, sum_s = 0.0;
       int64_t cnt_c = 0, cnt_s = 0;
       for (int64_t c = 0; c < block; ++c) {
         int64_t k = base + c;
         if (cat[r * K + k] == 2) continue;
         double aw = fabs((double)row[k]);
-        int sparse = split && (2.0 * aw > maxabs); /* |w| > 0.5 * max|w|  (R5) */
+        /* |w| > 0.5 * max|w| (R5), or |w| above the searched break-point */
+        int sparse = split == 2 ? (aw > pbest) : (split && (2.0 * aw > maxabs));
         cat[r * K + k] = sparse ? 1 : 0;
         b1[r * K + k] = (row[k] < 0.0f) ? -1 : 1;
         b2[r * K + k] = 0;

@@ -378,3 +378,59 @@ def test_attn_av_matches_dense_dequantized_product(orc):
     np.testing.assert_allclose(Oref, dense, rtol=1e-12, atol=1e-300)
     np.testing.assert_array_equal(O, np.einsum("hql,hdl->hqd", ap.astype(np.int64),
                                                av.reshape(BH, D, L).astype(np.int64)))
+
+
+# ------------------------------------------------ BiLLM break-point search
+def _frac(t):
+    a, b = t.split("/")
+    return float(a) / float(b)
+
+
+def test_billm_split_golden(orc):
+    for ws, mode, cats, ac, asp in read_golden("billm_split.txt"):
+        W = (np.array([float(v) for v in ws.split()], np.float32) / np.float32(128))[None, :]
+        sal = np.zeros((1, 0), np.int32)
+        q = orc.billm_quantize_rows(W, sal, 0, 1, block=8, split=int(mode))
+        assert q["cat"][0].tolist() == [int(v) for v in cats.split()], (ws, mode)
+        assert q["scales"][0, 0, 0] == np.float32(_frac(ac)), (ws, mode, q["scales"])
+        assert q["scales"][0, 0, 1] == np.float32(_frac(asp)), (ws, mode, q["scales"])
+
+
+def _np_split_error(v, p):
+    e = 0.0
+    for grp in (v[v <= p], v[v > p]):
+        if grp.size:
+            e += float(((grp - grp.mean()) ** 2).sum())
+    return e
+
+
+def test_billm_split_search_matches_numpy_brute_force(orc):
+    W = workloads.latent_laplace((12, 384), 0.01, 99, 12, 384)
+    sal = orc.billm_salient(W, 128, 8)
+    q = orc.billm_quantize_rows(W, sal, 0, 12, 128, split=2)
+    qf = orc.billm_quantize_rows(W, sal, 0, 12, 128, split=1)
+    for n in range(12):
+        for j in range(3):
+            cols = np.setdiff1d(np.arange(128), sal[j]) + 128 * j
+            v = np.abs(W[n, cols].astype(np.float64))
+            errs = [(_np_split_error(v, p), p) for p in np.unique(v)]
+            e_best, p_best = min(errs)      # ties: the smaller p
+            sparse = v > p_best
+            np.testing.assert_array_equal(q["cat"][n, cols] == 1, sparse)
+            ac = np.float32(v[~sparse].mean())
+            asp = np.float32(v[sparse].mean()) if sparse.any() else np.float32(0)
+            np.testing.assert_allclose(q["scales"][n, j, :2], [ac, asp], rtol=2 ** -23)
+            # the search never does worse than the fixed 0.5 * max break-point
+            fixed = v > 0.5 * v.max()
+            assert e_best <= _np_split_error(v, v[~fixed].max()) + 1e-18
+            assert (qf["cat"][n, cols] == 1).tolist() == fixed.tolist()
+
+
+def test_billm_split_search_lowers_reconstruction_error(orc):
+    W = workloads.latent_laplace((16, 256), 0.01, 98, 16, 256)
+    sal = orc.billm_salient(W, 128, 8)
+    e = {}
+    for mode in (0, 1, 2):
+        q = orc.billm_quantize_rows(W, sal, 0, 16, 128, split=mode)
+        e[mode] = float(((W.astype(np.float64) - orc.billm_dequant(q)) ** 2).sum())
+    assert e[2] <= e[1] <= e[0]
