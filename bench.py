@@ -3,9 +3,11 @@
 
 Default workload: the LLaMA-7B-shaped projections (K, N) in {(4096, 4096),
 (4096, 11008), (11008, 4096)} with per-128-column weight scales. One step =
-for each shape: ternarize+pack the decode activations (M=1) and run the GEMV,
-then ternarize+pack the prefill activations (M=2048) and run the tiled GEMM.
-Weights are binarized and packed once, before timing (an offline step).
+the decode phase (the three M=1 activation rows ternarized and multiplied by
+the three weight matrices in one fused launch), then for each shape: ternarize
+the prefill activations (M=2048, E4M3 bytes) and run the tensor-core GEMM.
+Weights are binarized and packed once, before timing (an offline step). The
+popcount GEMM on the same prefill products is timed beside the step.
 
 Metric: effective TOPS = sum over the step's products of 2*M*N*K, divided by
 the device time of the step (CUDA-graph replay, L2 flushed between steps by a
@@ -14,8 +16,9 @@ the device time of the step (CUDA-graph replay, L2 flushed between steps by a
 
 --impl reference times the CPU oracle (a plain C loop over unpacked values)
 on a bounded row sample of the same workload. --workload selects the other
-measured rows: llama_prefill, llama_decode, llama_decode_model, gemv_big, bert,
-tiny, attn, billm1, billm16, billm512, pack (comma separated, or all).
+measured rows: llama_prefill, llama_decode, llama_decode_batched,
+llama_decode_model, gemv_big, bert, tiny, attn, billm1, billm16, billm512, pack
+(comma separated, or all).
 """
 from __future__ import annotations
 
@@ -715,8 +718,8 @@ def run_rows(args):
     reps = max(3, args.steps)
     rows = args.workload.split(",")
     if "all" in rows:
-        rows = ["tiny", "bert", "llama_decode", "gemv_big", "llama_decode_model", "attn", "billm1",
-                "billm16", "billm512", "pack"]
+        rows = ["tiny", "bert", "llama_decode", "llama_decode_batched", "gemv_big",
+                "llama_decode_model", "attn", "billm1", "billm16", "billm512", "pack"]
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
     def emit(name, t, ops=None, nbytes=None, **extra):
@@ -761,6 +764,19 @@ def run_rows(args):
             for s in range(3):
                 t = workloads.llama(s, M)
                 linear_rows(f"llama{s}_{t['K']}x{t['N']}_M{M}", t["X"], t["W"], t["group"])
+        elif row == "llama_decode_batched":
+            jobs, nbytes, ops = [], 0, 0
+            for i in range(3):
+                t = workloads.llama(i, 1)
+                wb, ws = bt.bwta_pack_weights(dev(t["W"]), t["group"])
+                jobs.append((dev(t["X"]), wb, ws, t["group"]))
+                nbytes += wb.numel() * 4 + ws.numel() * 4 + t["K"] * 2 + t["N"] * 4
+                ops += 2 * t["N"] * t["K"]
+            desc = bt.decode_jobs(jobs)
+            t = _time_fn(lambda: bt.bwta_linear_decode_batched(
+                None, flags=bt.GEMM_WEIGHTS_READY, descriptors=desc), reps, flush)
+            emit("llama_decode_3_projections_one_launch", t, ops=ops, nbytes=nbytes,
+                 kernel="k_decode (fused ternarize + GEMV, 3 jobs)")
         elif row == "gemv_big":
             W = workloads.billm_weights()  # 28672 x 8192 latent weights, per-128 scales
             X = workloads.billm_acts(1)
@@ -780,6 +796,26 @@ def run_rows(args):
             Q, Kt = dev(a["Q"].reshape(-1, D)), dev(a["K"].reshape(-1, D))
             qm, qs, qsc = bt.bwta_quantize_pack_acts(Q)
             km, ks, ksc = bt.bwta_quantize_pack_acts(Kt)
+            # past the scores: ternary probabilities straight from the planes, then A . V
+            BH = B * H
+            pm, ps, psc = bt.bwta_attn_softmax_ternarize(qm, qs, qsc, km, ks, ksc, BH, L, L, D,
+                                                         1.0 / np.sqrt(D))
+            t = _time_fn(lambda: bt.bwta_attn_softmax_ternarize(
+                qm, qs, qsc, km, ks, ksc, BH, L, L, D, 1.0 / np.sqrt(D), out=(pm, ps, psc)),
+                reps, flush)
+            emit("attn_softmax_ternarize", t,
+                 nbytes=2 * (qm.numel() + km.numel()) * 4 + (qsc.numel() + ksc.numel()) * 4 +
+                 2 * pm.numel() * 4 + psc.numel() * 4,
+                 scores_per_s=round(BH * L * L / t / 1e9, 2), unit_note="G scores/s (fp64 softmax)")
+            V = workloads.attn_v()
+            Vt = dev(np.ascontiguousarray(V.reshape(BH, L, D).transpose(0, 2, 1)).reshape(-1, L))
+            vm, vs, vsc = bt.bwta_quantize_pack_acts(Vt)
+            O = torch.empty((BH, L, D), dtype=torch.float32, device="cuda")
+            t = _time_fn(lambda: bt.bwta_attn_av(pm, ps, psc, vm, vs, vsc, BH, L, D, L,
+                                                 out=(None, O)), reps, flush)
+            emit("attn_av", t, ops=2 * BH * L * L * D,
+                 nbytes=2 * (pm.numel() + vm.numel()) * 4 + (psc.numel() + vsc.numel()) * 4 +
+                 O.numel() * 4)
             t = _time_fn(lambda: bt.bwta_quantize_pack_acts(Q, out=(qm, qs, qsc)), reps, flush)
             emit("attn_quantize_pack_q", t, nbytes=Q.numel() * 2 + 2 * qm.numel() * 4 + qsc.numel() * 4)
             Si = torch.empty((B * H, L, L), dtype=torch.int32, device="cuda")
@@ -810,7 +846,9 @@ def run_rows(args):
                 emit(f"pack_weights_{K}x{N}", t, nbytes=W.numel() * 4 + W.numel() // 8 + W.numel() // 32)
             W = dev(workloads.billm_weights())
             t = _time_fn(lambda: bt.billm_pack_weights(W), 1, flush)
-            emit("billm_pack_weights", t, nbytes=W.numel() * 4)
+            emit("billm_pack_weights", t, nbytes=W.numel() * 4, split="0.5*max")
+            t = _time_fn(lambda: bt.billm_pack_weights(W, split=2), 1, flush)
+            emit("billm_pack_weights_searched_split", t, nbytes=W.numel() * 4, split="searched")
         else:
             raise SystemExit(f"unknown workload row {row}")
 

@@ -28,7 +28,8 @@ ERROR_NAMES = {1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA"}
 EXPORTS = ["bwta_pack_weights", "bwta_quantize_pack_acts", "bwta_quantize_pack_acts_ex",
            "bwta_gemm", "bwta_gemm_ex", "bwta_gemm_tc",
            "bwta_linear_decode", "bwta_attn_scores", "billm_pack_weights", "billm_gemm",
-           "bwta_linear_decode_batched", "bwta_selftest_gemm_timeout", "bwta_version"]
+           "bwta_linear_decode_batched", "bwta_attn_softmax_ternarize", "bwta_attn_av",
+           "bwta_selftest_gemm_timeout", "bwta_version"]
 GEMM_WEIGHTS_READY = 0x1
 
 
@@ -77,6 +78,9 @@ def load_library(path: str = LIB_PATH):
     lib.bwta_linear_decode.argtypes = [vp, i64, i64, i64, ci, cf, vp, vp, i64, i64, i64, vp, i64,
                                        vp, i64, C.c_uint32, vp, vp]
     lib.bwta_attn_scores.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp, vp]
+    lib.bwta_attn_softmax_ternarize.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                                cf, vp, vp, i64, vp, vp]
+    lib.bwta_attn_av.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp, vp]
     lib.billm_pack_weights.argtypes = [vp, i64, ci, C.POINTER(BillmWeightsC), vp, vp]
     lib.billm_gemm.argtypes = [vp, i64, i64, C.POINTER(BillmWeightsC), vp, i64, vp, vp]
     lib.bwta_linear_decode_batched.argtypes = [C.POINTER(DecodeJobC), i64, ci, cf, C.c_uint32, vp,
@@ -331,6 +335,44 @@ def bwta_attn_scores(q_mask, q_sign, q_scale, k_mask, k_sign, k_scale, BH: int, 
     return Si, Sf
 
 
+def bwta_attn_softmax_ternarize(q_mask, q_sign, q_scale, k_mask, k_sign, k_scale, BH: int,
+                                Lq: int, Lk: int, D: int, softmax_scale: float, out=None):
+    """Ternary attention probabilities from ternary Q, K planes (scores never
+    stored). Returns (p_mask, p_sign, p_scale): [BH*Lq, ld_words_for(Lk)] x2, [BH*Lq]."""
+    lib = _L()
+    ld = q_mask.shape[-1]
+    ldp = ld_words_for(Lk)
+    dev = q_mask.device
+    if out is None:
+        pm = torch.empty((BH * Lq, ldp), dtype=torch.int32, device=dev)
+        ps = torch.empty((BH * Lq, ldp), dtype=torch.int32, device=dev)
+        sc = torch.empty((BH * Lq,), dtype=torch.float32, device=dev)
+    else:
+        pm, ps, sc = out
+    _check("bwta_attn_softmax_ternarize", lib.bwta_attn_softmax_ternarize(
+        _ptr(q_mask), _ptr(q_sign), _ptr(q_scale), _ptr(k_mask), _ptr(k_sign), _ptr(k_scale),
+        BH, Lq, Lk, D, ld, softmax_scale, _ptr(pm), _ptr(ps), pm.shape[1], _ptr(sc), _stream()))
+    return pm, ps, sc
+
+
+def bwta_attn_av(p_mask, p_sign, p_scale, vt_mask, vt_sign, vt_scale, BH: int, Lq: int, D: int,
+                 Lk: int, want_int: bool = False, want_float: bool = True, out=None):
+    """A . V with ternary probabilities and V^T planes. Returns (O int32 or None,
+    O fp32 or None), each [BH, Lq, D]."""
+    lib = _L()
+    ld = p_mask.shape[-1]
+    dev = p_mask.device
+    if out is None:
+        Oi = torch.empty((BH, Lq, D), dtype=torch.int32, device=dev) if want_int else None
+        Of = torch.empty((BH, Lq, D), dtype=torch.float32, device=dev) if want_float else None
+    else:
+        Oi, Of = out
+    _check("bwta_attn_av", lib.bwta_attn_av(
+        _ptr(p_mask), _ptr(p_sign), _ptr(p_scale), _ptr(vt_mask), _ptr(vt_sign), _ptr(vt_scale),
+        BH, Lq, D, Lk, ld, _ptr(Oi), _ptr(Of), _stream()))
+    return Oi, Of
+
+
 # ------------------------------------------------------------------ BiLLM
 @dataclass
 class BillmWeights:
@@ -367,16 +409,17 @@ class BillmWeights:
             N=N, K=K, block=block, n_sal=n_sal)
 
 
-def billm_pack_weights(W: torch.Tensor, n_sal: int = 8, split: bool = True, block: int = 128,
+def billm_pack_weights(W: torch.Tensor, n_sal: int = 8, split=True, block: int = 128,
                        status=None) -> BillmWeights:
-    """Latent fp32 W [N, K] (cuda) -> packed BiLLM weights, built on the GPU."""
+    """Latent fp32 W [N, K] (cuda) -> packed BiLLM weights, built on the GPU.
+    split: False/0 no split, True/1 break-point 0.5*max|w|, 2 searched break-point."""
     lib = _L()
     assert W.is_cuda and W.dtype == torch.float32 and W.dim() == 2 and W.stride(1) == 1
     N, K = W.shape
     out = BillmWeights.empty(N, K, n_sal, block, W.device)
     cs = out.cstruct()
     _check("billm_pack_weights", lib.billm_pack_weights(
-        _ptr(W), _row_stride(W), int(bool(split)), C.byref(cs), _ptr(status), _stream()))
+        _ptr(W), _row_stride(W), int(split), C.byref(cs), _ptr(status), _stream()))
     return out
 
 

@@ -260,6 +260,38 @@ int bwta_attn_scores(const uint32_t *q_mask, const uint32_t *q_sign, const float
                                         Lk, D, ld_words, S_i32, S_f32, (cudaStream_t)stream));
 }
 
+int bwta_attn_softmax_ternarize(const uint32_t *q_mask, const uint32_t *q_sign,
+                                const float *q_scale, const uint32_t *k_mask,
+                                const uint32_t *k_sign, const float *k_scale, int64_t BH,
+                                int64_t Lq, int64_t Lk, int64_t D, int64_t ld_words,
+                                float softmax_scale, uint32_t *p_mask, uint32_t *p_sign,
+                                int64_t ldp_words, float *p_scale, bwta_stream_t stream) {
+  if (BH < 0 || Lq < 0 || Lk <= 0 || D <= 0) return BWTA_ERR_INVALID_ARG;
+  if (ld_words > 32 || !(softmax_scale == softmax_scale)) return BWTA_ERR_UNSUPPORTED;
+  if (attn_softmax_smem(Lk, ld_words) > 200 * 1024) return BWTA_ERR_UNSUPPORTED;
+  if (int r = check_plane(q_mask, BH * Lq, ld_words, D)) return r;
+  if (int r = check_plane(q_sign, BH * Lq, ld_words, D)) return r;
+  if (int r = check_plane(k_mask, BH * Lk, ld_words, D)) return r;
+  if (int r = check_plane(k_sign, BH * Lk, ld_words, D)) return r;
+  if (int r = check_plane(p_mask, BH * Lq, ldp_words, Lk)) return r;
+  if (int r = check_plane(p_sign, BH * Lq, ldp_words, Lk)) return r;
+  if (BH * Lq > 0 && (!q_scale || !p_scale)) return BWTA_ERR_INVALID_ARG;
+  if (BH > 0 && !k_scale) return BWTA_ERR_INVALID_ARG;
+  return cuda_status(launch_attn_softmax(q_mask, q_sign, q_scale, k_mask, k_sign, k_scale, BH, Lq,
+                                         Lk, D, ld_words, softmax_scale, p_mask, p_sign, ldp_words,
+                                         p_scale, (cudaStream_t)stream));
+}
+
+int bwta_attn_av(const uint32_t *p_mask, const uint32_t *p_sign, const float *p_scale,
+                 const uint32_t *vt_mask, const uint32_t *vt_sign, const float *vt_scale,
+                 int64_t BH, int64_t Lq, int64_t D, int64_t Lk, int64_t ld_words, int32_t *O_i32,
+                 float *O_f32, bwta_stream_t stream) {
+  // the ternary x ternary product of bwta_attn_scores with the probabilities
+  // as the query side and the channels of V as the key side
+  return bwta_attn_scores(p_mask, p_sign, p_scale, vt_mask, vt_sign, vt_scale, BH, Lq, D, Lk,
+                          ld_words, O_i32, O_f32, stream);
+}
+
 static int check_billm(const billm_weights *W) {
   if (!W) return BWTA_ERR_INVALID_ARG;
   if (W->N < 0 || W->K <= 0) return BWTA_ERR_INVALID_ARG;
@@ -277,6 +309,7 @@ int billm_pack_weights(const float *W, int64_t ldW, int split, const billm_weigh
                        int32_t *d_status, bwta_stream_t stream) {
   if (int r = check_billm(out)) return r;
   if (ldW < out->K || (out->N > 0 && !W)) return BWTA_ERR_INVALID_ARG;
+  if (split < 0 || split > 2) return BWTA_ERR_INVALID_ARG;
   if (out->N > 0 && (out->n_sal == 0 ? false : !out->sal)) return BWTA_ERR_INVALID_ARG;
   return cuda_status(launch_billm_pack(W, ldW, split, out, d_status, (cudaStream_t)stream));
 }

@@ -199,8 +199,11 @@ static cudaError_t launch_attn_nw(const uint32_t *qm, const uint32_t *qs, const 
 // memory. One CTA per (batch*head, 64 query rows) holds the head's K planes in
 // shared memory; a warp owns a query row: per key, the ternary dot, the fp32
 // score ((float)S * s_q) * s_k (the same value bwta_attn_scores writes) times
-// the softmax factor; then the row max, e = exp(x - max), the sum, p = e / sum,
-// the keep bits (one ballot per 32 keys is one mask word) and the kept sum.
+// the softmax factor (fp32); the row max; then in fp64 e = exp(x - max), the
+// sum, p = e / sum, the keep decision p > 1/(2 Lk) (one ballot per 32 keys is
+// one mask word) and the kept sum. fp64 keeps the decision and the scale
+// independent of the summation order: the ambiguity is confined to p within
+// ~1e-15 (relative) of the threshold.
 constexpr int AS_ROWS = 64, AS_THREADS = 256, AS_WARPS = AS_THREADS / 32;
 
 template <int NW>
@@ -215,7 +218,7 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
   uint4 *sKm = as_sm;
   uint4 *sKs = sKm + Lk * nc;
   float *sk = reinterpret_cast<float *>(sKs + Lk * nc);
-  float *xw = sk + Lk + (threadIdx.x / 32) * Lk;  // this warp's row of scores, then of exp
+  double *xw = reinterpret_cast<double *>(sk + ((Lk + 1) / 2) * 2) + (threadIdx.x / 32) * Lk;
   pdl_trigger();
   pdl_wait();
   const int64_t bh = blockIdx.y;
@@ -228,7 +231,7 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
   __syncthreads();
 
   const int w = threadIdx.x / 32, l = threadIdx.x % 32;
-  const float thr = 0.5f / (float)Lk;
+  const double thr = 0.5 / (double)Lk;
   for (int r = w; r < AS_ROWS; r += AS_WARPS) {
     const int64_t i = (int64_t)blockIdx.x * AS_ROWS + r;
     if (i >= Lq) break;
@@ -254,26 +257,26 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
           if (cc < nc) d += tern_dot<4>(qa[cc], qb[cc], sKm[j * nc + cc], sKs[j * nc + cc]);
       }
       const float x = ((__int2float_rn(d) * sqi) * sk[j]) * c;
-      xw[j] = x;
+      xw[j] = (double)x;
       mx = fmaxf(mx, x);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-    float z = 0.0f;
+    double z = 0.0;
     for (int64_t j = l; j < Lk; j += 32) {
-      const float e = expf(xw[j] - mx);
+      const double e = exp(xw[j] - (double)mx);
       xw[j] = e;
       z += e;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
     // keep bits: key j = 32t + l is bit l of mask word t
-    float ksum = 0.0f;
+    double ksum = 0.0;
     int kn = 0;
     uint32_t *mrow = pm + (bh * Lq + i) * ldp, *srow = ps + (bh * Lq + i) * ldp;
     for (int64_t t = 0; t * 32 < Lk; ++t) {
       const int64_t j = t * 32 + l;
-      const float p = j < Lk ? __fdiv_rn(xw[j], z) : 0.0f;
+      const double p = j < Lk ? __ddiv_rn(xw[j], z) : 0.0;
       const bool keep = p > thr;
       const uint32_t word = __ballot_sync(FULL, keep);
       if (keep) ksum += p;
@@ -292,13 +295,13 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
       ksum += __shfl_xor_sync(FULL, ksum, o);
       kn += __shfl_xor_sync(FULL, kn, o);
     }
-    if (l == 0) pscale[bh * Lq + i] = kn ? __fdiv_rn(ksum, (float)kn) : 0.0f;
+    if (l == 0) pscale[bh * Lq + i] = kn ? __double2float_rn(__ddiv_rn(ksum, (double)kn)) : 0.0f;
   }
 }
 
 size_t attn_softmax_smem(int64_t Lk, int64_t ld) {
   const int64_t nc = ld / 4 > 1 ? ld / 4 : 1;
-  return (size_t)Lk * nc * 32 + (size_t)Lk * 4 + (size_t)AS_WARPS * Lk * 4;
+  return (size_t)Lk * nc * 32 + (size_t)((Lk + 1) / 2) * 8 + (size_t)AS_WARPS * Lk * 8;
 }
 
 template <int NW>

@@ -70,9 +70,12 @@ bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, int elem_bytes, co
 // four K-words, broadcast for the rows and conflict-free for the columns thanks
 // to the swizzle. Per stage the CTA first
 // counts popc(mask) per (row, 4-word chunk) and stages the weight scales of
-// each chunk's group; at the end of every weight group each thread folds its
-// 64 integer dots into fp32 with acc = fma((float)d_g, alpha_g, acc), in group
-// order, and the epilogue multiplies by the activation scale.
+// each chunk's group (loaded into registers one k-tile ahead, so the staging
+// does not wait on global memory); at the end of every weight group each
+// thread folds its 32 integer dots into fp32 with acc = fma((float)d_g,
+// alpha_g, acc), in group order, and the epilogue multiplies by the
+// activation scale. With 128-column groups (G1: every chunk is a group) a
+// chunk's dot goes straight into that fold, with no integer accumulator.
 constexpr int GM_BM = 128, GM_BN = 128, GM_BKW = 32, GM_STAGES = 3, GM_THREADS = 512;
 constexpr int GM_TI = 8, GM_TJ = 4;  // outputs per thread: rows ty + 16*i, columns tx + 32*j
 constexpr int GM_CHUNKS = GM_BKW / 4;
@@ -81,7 +84,7 @@ constexpr int GM_TILE_BYTES = GM_TILE_WORDS * 4;
 constexpr size_t GM_SMEM = 1024 + (size_t)GM_STAGES * 3 * GM_TILE_BYTES +
                            2 * GM_CHUNKS * GM_BM * 4 + (GM_STAGES + 1) * 8;
 
-template <bool GROUPED, bool WANT_Y, bool WANT_DOTS>
+template <bool GROUPED, bool WANT_Y, bool WANT_DOTS, bool G1>
 __global__ void __launch_bounds__(GM_THREADS, 1)
 k_gemm_tiled(const __grid_constant__ CUtensorMap map_am, const __grid_constant__ CUtensorMap map_as,
              const __grid_constant__ CUtensorMap map_w, const float *__restrict__ ascale,
@@ -89,6 +92,7 @@ k_gemm_tiled(const __grid_constant__ CUtensorMap map_am, const __grid_constant__
              int64_t G, float *__restrict__ Y, int64_t ldY, int32_t *__restrict__ dots,
              int64_t ldD, int32_t *d_status, uint64_t stall_ns) {
   static_assert(!(GROUPED && WANT_DOTS), "grouped dots come from the ungrouped pass");
+  static_assert(!G1 || GROUPED, "G1 is the grouped kernel with one chunk per group");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -139,6 +143,21 @@ k_gemm_tiled(const __grid_constant__ CUtensorMap map_am, const __grid_constant__
       y[i][j] = 0.0f;
     }
   }
+  // this thread's weight scales of the next k-tile: entries idx = tid + 512 q
+  // of the [chunk][weight row] staging table
+  constexpr int AQ = GM_CHUNKS * GM_BN / GM_THREADS;
+  float anext[AQ];
+  auto load_scales = [&](int kt) {
+#pragma unroll
+    for (int q = 0; q < AQ; ++q) {
+      const int idx = tid + GM_THREADS * q, c = idx >> 7, r = idx & 127;
+      const int gc = kt * GM_CHUNKS + c;
+      const int64_t n = n0 + r;
+      anext[q] = (GROUPED && kt < KT && gc < nchunks && n < N) ? __ldg(wscale + n * G + gc / gchunks)
+                                                               : 0.0f;
+    }
+  };
+  if (GROUPED) load_scales(0);
 
   for (int kt = 0; kt < KT; ++kt) {
     const int st = kt % GM_STAGES;
@@ -162,14 +181,42 @@ k_gemm_tiled(const __grid_constant__ CUtensorMap map_am, const __grid_constant__
       const int c = idx >> 7, r = idx & 127;
       const uint4 v = *reinterpret_cast<const uint4 *>(Am + swz128(r, c));
       Pst[idx] = __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
-      if (GROUPED) {
-        const int gc = kt * GM_CHUNKS + c;
-        const int64_t n = n0 + r;
-        Ast[idx] = (gc < nchunks && n < N) ? __ldg(wscale + n * G + gc / gchunks) : 0.0f;
-      }
+    }
+    if (GROUPED) {
+#pragma unroll
+      for (int q = 0; q < AQ; ++q) Ast[tid + GM_THREADS * q] = anext[q];
     }
     __syncthreads();
+    if (GROUPED) load_scales(kt + 1);  // in flight while this k-tile is computed
     const int cmax = min(GM_CHUNKS, nchunks - kt * GM_CHUNKS);
+    if (G1) {
+      // every chunk is a weight group: its dot goes straight into the fold
+      for (int c = 0; c < cmax; ++c) {
+        uint4 wv[GM_TJ];
+        float a[GM_TJ];
+#pragma unroll
+        for (int j = 0; j < GM_TJ; ++j) {
+          wv[j] = *reinterpret_cast<const uint4 *>(Wt + swz128(tx + 32 * j, c));
+          a[j] = Ast[c * GM_BN + tx + 32 * j];
+        }
+#pragma unroll
+        for (int i = 0; i < GM_TI; ++i) {
+          const int r = ty + 16 * i;
+          const uint4 am = *reinterpret_cast<const uint4 *>(Am + swz128(r, c));
+          const uint4 as = *reinterpret_cast<const uint4 *>(As + swz128(r, c));
+          const int pb = (int)Pst[c * GM_BM + r] + INT_FLOAT_BIAS;
+#pragma unroll
+          for (int j = 0; j < GM_TJ; ++j) {
+            const int cnt = popc4_csa(lop3_and_xor(am.x, as.x, wv[j].x), lop3_and_xor(am.y, as.y, wv[j].y),
+                                      lop3_and_xor(am.z, as.z, wv[j].z), lop3_and_xor(am.w, as.w, wv[j].w));
+            y[i][j] = fmaf(biased_int_to_float(pb - 2 * cnt), a[j], y[i][j]);
+          }
+        }
+      }
+      __syncthreads();
+      if (tid == 0 && kt + GM_STAGES < KT) issue(kt + GM_STAGES, st);
+      continue;
+    }
     for (int c = 0; c < cmax; ++c) {
       uint4 wv[GM_TJ];
 #pragma unroll
@@ -231,13 +278,13 @@ k_gemm_tiled(const __grid_constant__ CUtensorMap map_am, const __grid_constant__
   }
 }
 
-template <bool GROUPED, bool WANT_Y, bool WANT_DOTS>
+template <bool GROUPED, bool WANT_Y, bool WANT_DOTS, bool G1 = false>
 static cudaError_t launch_tiled_t(const CUtensorMap &mam, const CUtensorMap &mas,
                                   const CUtensorMap &mw, const float *ascale, const float *wscale,
                                   int64_t M, int64_t N, int nchunks, int gchunks, int64_t G,
                                   float *Y, int64_t ldY, int32_t *dots, int64_t ldD,
                                   int32_t *d_status, uint64_t stall_ns, cudaStream_t s) {
-  auto kern = k_gemm_tiled<GROUPED, WANT_Y, WANT_DOTS>;
+  auto kern = k_gemm_tiled<GROUPED, WANT_Y, WANT_DOTS, G1>;
   static SmemOptIn opt_in;
   if (cudaError_t e = opt_in(kern, (int)GM_SMEM)) return e;
   dim3 grid((unsigned)ceil_div<int64_t>(N, GM_BN), (unsigned)ceil_div<int64_t>(M, GM_BM));
@@ -270,7 +317,10 @@ cudaError_t launch_gemm_tiled(const uint32_t *am, const uint32_t *as, const floa
   const int gchunks = (int)(group / 128);
   const int64_t G = ceil_div<int64_t>(K, group);
   cudaError_t e = cudaSuccess;
-  if (Y)
+  if (Y && gchunks == 1)
+    e = launch_tiled_t<true, true, false, true>(mam, mas, mw, ascale, wscale, M, N, nchunks, gchunks,
+                                                G, Y, ldY, nullptr, ldD, d_status, stall_ns, s);
+  else if (Y)
     e = launch_tiled_t<true, true, false>(mam, mas, mw, ascale, wscale, M, N, nchunks, gchunks, G,
                                           Y, ldY, nullptr, ldD, d_status, stall_ns, s);
   if (e == cudaSuccess && dots)  // full-K integer dots: the same kernel without groups

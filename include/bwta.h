@@ -237,6 +237,52 @@ int bwta_attn_scores(const uint32_t *q_mask, const uint32_t *q_sign, const float
                      int64_t BH, int64_t Lq, int64_t Lk, int64_t D, int64_t ld_words,
                      int32_t *S_i32, float *S_f32, bwta_stream_t stream);
 
+/* Attention probabilities as ternary planes, straight from the ternary Q and
+ * K planes (BWTA abstract: binary/ternary MatMul for the attention operators;
+ * the probabilities are the activations of the A . V product and are
+ * ternarized like any activation). Per query row i of each batch*head, over
+ * the Lk keys j:
+ *   x_ij = (((float)S_ij * q_scale_i) * k_scale_j) * softmax_scale   (S as in
+ *          bwta_attn_scores; the score before the factor is the fp32 value that
+ *          bwta_attn_scores writes)
+ *   p_ij = exp(x_ij - max_j x) / sum_j exp(x_ij - max_j x)   (fp64, from the fp32 x)
+ *   kept iff p_ij > 0.5 * mean_j p_ij, where the mean of a softmax row is
+ *   exactly 1/Lk, so kept iff p_ij > 1/(2 Lk); every p is positive, so a kept
+ *   value is +1 and the sign plane is all zero; p_scale_i = mean of the kept p.
+ * The Lq x Lk scores are never written to memory. The kept decision and the
+ * scale are taken in fp64, so they do not depend on the order of the sums; a
+ * probability within about 1e-15 (relative) of 1/(2 Lk) can fall either way.
+ *  q_*, k_*, BH, Lq, Lk, D, ld_words   as bwta_attn_scores (ld_words <= 32)
+ *  p_mask, p_sign  uint32 [BH*Lq][ldp_words] out (ldp_words >= ceil(Lk/32),
+ *                  % 4 == 0; padding words written as zero)
+ *  p_scale         fp32 [BH*Lq] out
+ *  Limits: Lk * (32 * ceil(ld_words/4) + 68) bytes <= 200 KB (shared memory).
+ *  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA. */
+int bwta_attn_softmax_ternarize(const uint32_t *q_mask, const uint32_t *q_sign,
+                                const float *q_scale, const uint32_t *k_mask,
+                                const uint32_t *k_sign, const float *k_scale, int64_t BH,
+                                int64_t Lq, int64_t Lk, int64_t D, int64_t ld_words,
+                                float softmax_scale, uint32_t *p_mask, uint32_t *p_sign,
+                                int64_t ldp_words, float *p_scale, bwta_stream_t stream);
+
+/* The A . V product of attention with ternary operands (BWTA abstract:
+ * binary/ternary MatMul for the attention operators): the ternary
+ * probabilities from bwta_attn_softmax_ternarize times V, ternarized per
+ * output channel over the sequence (bwta_quantize_pack_acts on the rows of
+ * V^T, so that each channel's scale factors out of the sum over keys):
+ *   O_i32[h][i][d] = sum_j p_ij * v_dj   (p in {0, 1}, v in {-1, 0, 1})
+ *   O_f32[h][i][d] = ((float)O_i32 * p_scale[h][i]) * v_scale[h][d]
+ *  p_mask, p_sign, p_scale   [BH*Lq][ld_words], [BH*Lq]
+ *  vt_mask, vt_sign, vt_scale [BH*D][ld_words], [BH*D]: row d of head h is
+ *                  channel d of V over the Lk keys
+ *  ld_words        >= ceil(Lk/32), % 4 == 0, the same for both sides
+ *  O_i32, O_f32    [BH][Lq][D] out, either may be NULL (not both)
+ *  Errors: INVALID_ARG, UNSUPPORTED (ld_words > 32), ALIGNMENT, CUDA. */
+int bwta_attn_av(const uint32_t *p_mask, const uint32_t *p_sign, const float *p_scale,
+                 const uint32_t *vt_mask, const uint32_t *vt_sign, const float *vt_scale,
+                 int64_t BH, int64_t Lq, int64_t D, int64_t Lk, int64_t ld_words, int32_t *O_i32,
+                 float *O_f32, bwta_stream_t stream);
+
 /* BiLLM packed weights (BiLLM "Approach" and "Limitations"). Per block j of
  * `block` = 128 columns and row n:
  *  sign   uint32 [N][ldw_words]  1 = negative (b for non-salient, b1 for salient)
@@ -260,11 +306,16 @@ typedef struct billm_weights {
  *  (fp64, rows ascending; the Hessian of the pages' metric taken as the
  *  identity, as no calibration data is used); ties go to the lower column.
  *  Salient weights: alpha1 = mean|w|, b1 = sign(w), r = w - alpha1*b1,
- *  alpha2 = mean|r|, b2 = sign(r). Other weights: break-point
- *  p = 0.5*max|w| over the row's non-salient weights in the block; the sparse
- *  group is |w| > p (only if split != 0); alpha = mean|w| per group (0 if
- *  empty). Every mean is an fp64 sum in ascending column order divided by the
- *  count and rounded once to fp32.
+ *  alpha2 = mean|r|, b2 = sign(r). Other weights: a break-point p per row
+ *  and block, the sparse group is |w| > p; split selects p:
+ *    0  no split (every non-salient weight is concentrated)
+ *    1  p = 0.5*max|w| over the row's non-salient weights in the block
+ *    2  the searched break-point (BiLLM abstract: "optimal splitting search"):
+ *       the non-salient magnitude of the row-block whose split minimizes the
+ *       squared binarization error sum (|w| - alpha_group)^2 of both groups,
+ *       evaluated in fp64 in ascending column order; ties go to the smaller p
+ *  alpha = mean|w| per group (0 if empty). Every mean is an fp64 sum in
+ *  ascending column order divided by the count and rounded once to fp32.
  *  W fp32 [N][ldW]; out: the buffers of `out` (cast away const; device memory).
  *  block must be 128; 0 <= n_sal <= 8; K % 128 == 0.
  *  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; NONFINITE flag. */

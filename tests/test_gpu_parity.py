@@ -356,7 +356,7 @@ def billm_rows_ref(X, W, sal, rows, split=True):
 
 @pytest.mark.parametrize("N,K,M,n_sal,split", [
     (40, 384, 3, 8, True), (33, 256, 17, 8, True), (70, 512, 1, 0, False), (64, 1024, 5, 3, True),
-    (100, 128, 40, 8, False)])
+    (100, 128, 40, 8, False), (40, 384, 1, 8, 2), (50, 256, 20, 0, 2), (33, 512, 3, 3, 2)])
 def test_billm_small(N, K, M, n_sal, split):
     W = workloads.latent_laplace((N, K), 0.01, 7, N, K)
     X = workloads.edge_acts(M, K, "normal", tag=N)
@@ -385,6 +385,21 @@ def test_billm_full_config(billm_full, M):
     Y = bt.billm_gemm(dev(X), Wq).cpu().numpy()
     yref, mag = billm_rows_ref(X, W, sal, rows)
     assert_close_rel(Y[:, rows], yref, mag, what=f"billm M={M}")
+
+
+def test_billm_searched_split_full_config_rows():
+    """The searched break-point (split = 2) on the BiLLM configuration: packed
+    planes, residual bits and scales equal the oracle's bit for bit on sampled
+    rows, and the GEMM on those weights matches the oracle."""
+    W = workloads.billm_weights()
+    Wq = bt.billm_pack_weights(dev(W), split=2)
+    torch.cuda.synchronize()
+    rows = sample_rows(W.shape[0], 16)
+    sal, _ = check_billm_pack(W, Wq, rows, 8, 2)
+    X = workloads.billm_acts(1)
+    Y = bt.billm_gemm(dev(X), Wq).cpu().numpy()
+    yref, mag = billm_rows_ref(X, W, sal, rows, split=2)
+    assert_close_rel(Y[:, rows], yref, mag, what="billm searched split")
 
 
 @pytest.mark.parametrize("N,K,M", [(200, 384, 300), (129, 128, 70), (64, 1024, 2), (300, 256, 257)])

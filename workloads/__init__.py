@@ -16,7 +16,7 @@ distributions follow the workloads the library is measured on:
   at M = 2048 (prefill) and M = 1 (decode); W ~ N(0, 0.02); X ~ Student-t(nu=3)
   with 1% of the entries (Bernoulli per element) multiplied by 20, clipped to
   the fp16 range
-* attention scores: Q, K of shape [8, 12, 512, 64] ~ N(0, 1)
+* attention: Q, K, V of shape [8, 12, 512, 64] ~ N(0, 1)
 * BiLLM-format GEMM at the LLaMA-2-70B FFN shape: K=8192, N=28672,
   W ~ Laplace(0, 0.01), X ~ N(0, 1) at M in {1, 16, 512}
 """
@@ -103,6 +103,11 @@ def attn(shape=ATTN_SHAPE):
     Q = acts_normal(shape, CFG_ATTN, 0, *shape)
     Kt = acts_normal(shape, CFG_ATTN, 1, *shape)
     return dict(Q=Q, K=Kt)
+
+
+def attn_v(shape=ATTN_SHAPE):
+    """V of the attention workload, [batch, heads, seq, head_dim] ~ N(0, 1)."""
+    return acts_normal(shape, CFG_ATTN, 2, *shape)
 
 
 def billm_weights(N: int = BILLM_N, K: int = BILLM_K):
