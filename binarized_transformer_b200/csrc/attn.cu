@@ -87,13 +87,17 @@ k_attn_scores(const uint32_t *__restrict__ qm, const uint32_t *__restrict__ qs,
     sQm[idx] = in ? __ldg(reinterpret_cast<const uint4 *>(qm + off) + c) : z4;
     sQs[idx] = in ? __ldg(reinterpret_cast<const uint4 *>(qs + off) + c) : z4;
   }
+  // K tile: [key][chunk] for one-chunk rows; chunk-major [chunk][key] for the
+  // general path, so that lanes reading consecutive keys hit consecutive
+  // 16-byte slots (no bank conflicts)
   for (int idx = threadIdx.x; idx < AT_TK * nc; idx += AT_THREADS) {
     const int r = idx / nc, c = idx % nc;
     const int64_t j = j0 + r;
     const bool in = j < Lk;
     const int64_t off = (bh * Lk + j) * ld;
-    sKm[idx] = in ? __ldg(reinterpret_cast<const uint4 *>(km + off) + c) : z4;
-    sKs[idx] = in ? __ldg(reinterpret_cast<const uint4 *>(ks + off) + c) : z4;
+    const int dst = NW == 4 ? c * AT_TK + r : idx;
+    sKm[dst] = in ? __ldg(reinterpret_cast<const uint4 *>(km + off) + c) : z4;
+    sKs[dst] = in ? __ldg(reinterpret_cast<const uint4 *>(ks + off) + c) : z4;
   }
   if (WF) {
     for (int idx = threadIdx.x; idx < AT_TQ; idx += AT_THREADS)
@@ -104,10 +108,13 @@ k_attn_scores(const uint32_t *__restrict__ qm, const uint32_t *__restrict__ qs,
   __syncthreads();
 
   const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  // this lane's keys: 4l .. 4l+3 (one-chunk rows, one 16-byte store per row)
+  // or l, l+32, l+64, l+96 (general path, four coalesced 4-byte stores)
+  auto key = [&](int t) { return NW == 4 ? l + 32 * t : 4 * l + t; };
   const int64_t jb = j0 + 4 * l;
   float skv[4];
 #pragma unroll
-  for (int t = 0; t < 4; ++t) skv[t] = WF ? sk[4 * l + t] : 0.0f;
+  for (int t = 0; t < 4; ++t) skv[t] = WF ? sk[key(t)] : 0.0f;
   uint4 kmv[4], ksv[4];
   if (NW != 4) {
 #pragma unroll
@@ -129,16 +136,26 @@ k_attn_scores(const uint32_t *__restrict__ qm, const uint32_t *__restrict__ qs,
         const uint4 a = sQm[r * nc + c], b = sQs[r * nc + c];
 #pragma unroll
         for (int t = 0; t < 4; ++t)
-          d[t] += tern_dot<4>(a, b, sKm[(4 * l + t) * nc + c], sKs[(4 * l + t) * nc + c]);
+          d[t] += tern_dot<4>(a, b, sKm[c * AT_TK + key(t)], sKs[c * AT_TK + key(t)]);
       }
     }
-    const int64_t o = (bh * Lq + i) * Lk + jb;
     float f[4];
     if (WF) {
       const float sqi = sq[r];
 #pragma unroll
       for (int t = 0; t < 4; ++t) f[t] = (__int2float_rn(d[t]) * sqi) * skv[t];
     }
+    if (NW == 4) {
+      const int64_t orow = (bh * Lq + i) * Lk + j0;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        if (j0 + key(t) >= Lk) break;
+        if (WI) __stcs(Si + orow + key(t), d[t]);
+        if (WF) __stcs(Sf + orow + key(t), f[t]);
+      }
+      continue;
+    }
+    const int64_t o = (bh * Lq + i) * Lk + jb;
     if (VEC && jb + 3 < Lk) {
       if (WI) st_cs(Si + o, make_int4(d[0], d[1], d[2], d[3]));
       if (WF) st_cs(Sf + o, make_float4(f[0], f[1], f[2], f[3]));
@@ -199,11 +216,13 @@ static cudaError_t launch_attn_nw(const uint32_t *qm, const uint32_t *qs, const 
 // memory. One CTA per (batch*head, 64 query rows) holds the head's K planes in
 // shared memory; a warp owns a query row: per key, the ternary dot, the fp32
 // score ((float)S * s_q) * s_k (the same value bwta_attn_scores writes) times
-// the softmax factor (fp32); the row max; then in fp64 e = exp(x - max), the
-// sum, p = e / sum, the keep decision p > 1/(2 Lk) (one ballot per 32 keys is
-// one mask word) and the kept sum. fp64 keeps the decision and the scale
-// independent of the summation order: the ambiguity is confined to p within
-// ~1e-15 (relative) of the threshold.
+// the softmax factor (fp32); the row max; e = exp(x - max) in fp32 (the CUDA
+// expf, a few ulp); then in fp64 the sum Z, the keep decision e > Z / (2 Lk)
+// (that is p = e / Z > 1/(2 Lk), without a divide per key; one ballot per 32
+// keys is one mask word) and the kept sum. The fp64 sums make the decision and
+// the scale independent of the summation order; what remains is expf's
+// rounding, so a probability within ~1e-6 (relative) of the threshold can
+// fall either way.
 constexpr int AS_ROWS = 64, AS_THREADS = 256, AS_WARPS = AS_THREADS / 32;
 
 template <int NW>
@@ -218,7 +237,7 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
   uint4 *sKm = as_sm;
   uint4 *sKs = sKm + Lk * nc;
   float *sk = reinterpret_cast<float *>(sKs + Lk * nc);
-  double *xw = reinterpret_cast<double *>(sk + ((Lk + 1) / 2) * 2) + (threadIdx.x / 32) * Lk;
+  float *xw = sk + Lk + (threadIdx.x / 32) * Lk;  // this warp's row of scores, then of exp
   pdl_trigger();
   pdl_wait();
   const int64_t bh = blockIdx.y;
@@ -231,7 +250,7 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
   __syncthreads();
 
   const int w = threadIdx.x / 32, l = threadIdx.x % 32;
-  const double thr = 0.5 / (double)Lk;
+  const double thr = 0.5 / (double)Lk;  // the keep test e > Z * thr
   for (int r = w; r < AS_ROWS; r += AS_WARPS) {
     const int64_t i = (int64_t)blockIdx.x * AS_ROWS + r;
     if (i >= Lq) break;
@@ -257,33 +276,39 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
           if (cc < nc) d += tern_dot<4>(qa[cc], qb[cc], sKm[j * nc + cc], sKs[j * nc + cc]);
       }
       const float x = ((__int2float_rn(d) * sqi) * sk[j]) * c;
-      xw[j] = (double)x;
+      xw[j] = x;
       mx = fmaxf(mx, x);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
     double z = 0.0;
     for (int64_t j = l; j < Lk; j += 32) {
-      const double e = exp(xw[j] - (double)mx);
+      const float e = expf(xw[j] - mx);
       xw[j] = e;
-      z += e;
+      z += (double)e;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
+    const double cut = z * thr;
     // keep bits: key j = 32t + l is bit l of mask word t
     double ksum = 0.0;
     int kn = 0;
     uint32_t *mrow = pm + (bh * Lq + i) * ldp, *srow = ps + (bh * Lq + i) * ldp;
+    uint32_t myword = 0;  // lane l keeps mask word l (of each group of 32 words)
     for (int64_t t = 0; t * 32 < Lk; ++t) {
       const int64_t j = t * 32 + l;
-      const double p = j < Lk ? __ddiv_rn(xw[j], z) : 0.0;
-      const bool keep = p > thr;
+      const double e = j < Lk ? (double)xw[j] : 0.0;
+      const bool keep = e > cut;
       const uint32_t word = __ballot_sync(FULL, keep);
-      if (keep) ksum += p;
+      if (keep) ksum += e;
       kn += keep;
-      if (l == 0) {
-        mrow[t] = word;
-        srow[t] = 0u;
+      if (l == (t & 31)) myword = word;
+      if ((t & 31) == 31 || (t + 1) * 32 >= Lk) {  // one coalesced store per 32 words
+        const int64_t t0 = t & ~(int64_t)31;
+        if (t0 + l <= t) {
+          mrow[t0 + l] = myword;
+          srow[t0 + l] = 0u;
+        }
       }
     }
     for (int t = (int)((Lk + 31) / 32) + l; t < ldp; t += 32) {  // padding words
@@ -295,13 +320,14 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
       ksum += __shfl_xor_sync(FULL, ksum, o);
       kn += __shfl_xor_sync(FULL, kn, o);
     }
-    if (l == 0) pscale[bh * Lq + i] = kn ? __double2float_rn(__ddiv_rn(ksum, (double)kn)) : 0.0f;
+    // scale = mean of the kept p = (sum of the kept e / Z) / count
+    if (l == 0) pscale[bh * Lq + i] = kn ? __double2float_rn(__ddiv_rn(__ddiv_rn(ksum, z), (double)kn)) : 0.0f;
   }
 }
 
 size_t attn_softmax_smem(int64_t Lk, int64_t ld) {
   const int64_t nc = ld / 4 > 1 ? ld / 4 : 1;
-  return (size_t)Lk * nc * 32 + (size_t)((Lk + 1) / 2) * 8 + (size_t)AS_WARPS * Lk * 8;
+  return (size_t)Lk * nc * 32 + (size_t)Lk * 4 + (size_t)AS_WARPS * Lk * 4;
 }
 
 template <int NW>

@@ -80,32 +80,52 @@ k_billm_salient(const float *__restrict__ W, int64_t N, int64_t ldW, int n_sal,
 // (a = the group's mean magnitude, its L2-optimal scale) wins; ties go to the
 // smaller p. E is evaluated in fp64 in ascending column order with explicit
 // round-to-nearest operations (no fused multiply-add), so the decision is the
-// same on every run.
-__device__ double billm_split_error(const float *__restrict__ wr, const uint32_t (&salmask)[4],
-                                   double p) {
-  double sc = 0.0, ss = 0.0;
-  int nc = 0, ns = 0;
+// same on every run; eight candidates share each pass over the columns.
+// E(p) of eight candidate break-points at once: eight independent fp64
+// chains per pass over the columns (the same operations, in the same column
+// order, as one candidate at a time). Salient columns and candidates past the
+// last one (cand[u] < 0) contribute nothing.
+__device__ __forceinline__ void billm_split_errors8(const float *__restrict__ wr, const uint32_t (&salmask)[4],
+                                    const double (&p)[8], double (&e)[8]) {
+  double sc[8], ss[8];
+  int nc[8], ns[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    sc[u] = ss[u] = 0.0;
+    nc[u] = ns[u] = 0;
+  }
   for (int c = 0; c < 128; ++c) {
-    if ((salmask[c >> 5] >> (c & 31)) & 1u) continue;
+    if ((salmask[c >> 5] >> (c & 31)) & 1u) continue;  // the same for all eight
     const double aw = fabs((double)__ldg(wr + c));
-    if (aw <= p) {
-      sc = __dadd_rn(sc, aw);
-      ++nc;
-    } else {
-      ss = __dadd_rn(ss, aw);
-      ++ns;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (aw <= p[u]) {
+        sc[u] = __dadd_rn(sc[u], aw);
+        ++nc[u];
+      } else {
+        ss[u] = __dadd_rn(ss[u], aw);
+        ++ns[u];
+      }
     }
   }
-  const double ac = nc ? __ddiv_rn(sc, (double)nc) : 0.0, as = ns ? __ddiv_rn(ss, (double)ns) : 0.0;
-  double e = 0.0;
+  double ac[8], as[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    ac[u] = nc[u] ? __ddiv_rn(sc[u], (double)nc[u]) : 0.0;
+    as[u] = ns[u] ? __ddiv_rn(ss[u], (double)ns[u]) : 0.0;
+    e[u] = 0.0;
+  }
   for (int c = 0; c < 128; ++c) {
     if ((salmask[c >> 5] >> (c & 31)) & 1u) continue;
     const double aw = fabs((double)__ldg(wr + c));
-    const double d = __dsub_rn(aw, aw <= p ? ac : as);
-    e = __dadd_rn(e, __dmul_rn(d, d));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const double d = __dsub_rn(aw, aw <= p[u] ? ac[u] : as[u]);
+      e[u] = __dadd_rn(e[u], __dmul_rn(d, d));
+    }
   }
-  return e;
 }
+
 __global__ void __launch_bounds__(256)
 k_billm_quantize(const float *__restrict__ W, int64_t N, int64_t K, int64_t ldW, int n_sal,
                  int split, const uint8_t *__restrict__ sal, uint32_t *__restrict__ sign,
@@ -146,15 +166,30 @@ k_billm_quantize(const float *__restrict__ W, int64_t N, int64_t K, int64_t ldW,
     if (!((salmask[c >> 5] >> (c & 31)) & 1u)) maxabs = fmax(maxabs, fabs((double)__ldg(wr + c)));
   double pbest = maxabs;
   if (split == 2) {
+    // candidates: the non-salient magnitudes, eight per pass over the columns
     double ebest = __longlong_as_double(0x7ff0000000000000LL);  // +inf
-    for (int c0 = 0; c0 < 128; ++c0) {
-      if ((salmask[c0 >> 5] >> (c0 & 31)) & 1u) continue;
-      const double p = fabs((double)__ldg(wr + c0));
-      const double e = billm_split_error(wr, salmask, p);
-      if (e < ebest || (e == ebest && p < pbest)) {
-        ebest = e;
-        pbest = p;
+    int c0 = 0;
+    while (c0 < 128) {
+      double p[8], e[8];
+      bool v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {  // the next eight non-salient columns
+        while (c0 < 128 && ((salmask[c0 >> 5] >> (c0 & 31)) & 1u)) ++c0;
+        v[u] = c0 < 128;
+        p[u] = v[u] ? fabs((double)__ldg(wr + c0)) : 0.0;
+        if (v[u]) ++c0;
       }
+      if (!v[0]) break;
+#pragma unroll
+      for (int u = 1; u < 8; ++u)
+        if (!v[u]) p[u] = p[0];  // padding: repeats a candidate
+      billm_split_errors8(wr, salmask, p, e);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (v[u] && (e[u] < ebest || (e[u] == ebest && p[u] < pbest))) {
+          ebest = e[u];
+          pbest = p[u];
+        }
     }
   }
   double sc = 0.0, ss = 0.0;
@@ -393,154 +428,6 @@ k_billm_rows(const uint16_t *__restrict__ X, int64_t M, int64_t ldX, const uint3
   if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
 }
 
-// ------------------------------------------------------------ M = 1 (decode)
-// One activation row. Per slice of K (up to 4096 columns) the CTA builds a
-// table of subset sums: for every 4-column nibble q and every pattern p of its
-// four bits, L[q][p] = sum of x[4q + i] over the set bits i of p (fp32, i
-// ascending). The sum of x over a row-block's negative-sign columns is then one
-// table lookup and one add per nibble -- a quarter of a lookup per weight --
-// instead of one predicated add per weight; the one-bit entries L[q][1 << i]
-// are the x values the sparse and salient corrections need, and the block sums
-// X_j = sum_c x[c] come from the all-ones entries. Threads and blocks are laid
-// out as in k_billm_rows (four threads per weight row on interleaved blocks).
-constexpr int BL_SLICE = 4096;
-constexpr int BL_BSTRIDE = 32 * 16 + 4;  // floats per block of 32 nibbles (the pad spreads banks)
-
-__global__ void __launch_bounds__(BR_THREADS)
-k_billm_gemv_lut(const uint16_t *__restrict__ X, const uint32_t *__restrict__ sign,
-                 const uint32_t *__restrict__ gmap, const uint8_t *__restrict__ res,
-                 const uint8_t *__restrict__ sal, const float *__restrict__ bscale, int64_t N,
-                 int64_t K, int64_t ldw, int n_sal, float *__restrict__ Y, int32_t *d_status) {
-  extern __shared__ float4 bl_smem4[];
-  float *lut = reinterpret_cast<float *>(bl_smem4);              // [BL_SLICE / 128][BL_BSTRIDE]
-  float *xsum = lut + (BL_SLICE / 128) * BL_BSTRIDE;             // [BL_SLICE / 128]
-  uint8_t *ssal = reinterpret_cast<uint8_t *>(xsum + BL_SLICE / 128);  // [nb][n_sal]
-  pdl_trigger();
-  pdl_wait();
-  const int nb = (int)(K / 128);
-  for (int i = threadIdx.x; i < nb * n_sal; i += BR_THREADS) ssal[i] = sal[i];
-  const int lane = threadIdx.x % 32, part = lane % BR_SPLIT;
-  const int slot = (threadIdx.x / 32) * (32 / BR_SPLIT) + lane / BR_SPLIT;
-  const int64_t groups = ceil_div<int64_t>(N, BR_ROWS);
-  bool bad = false;
-  for (int64_t rg = blockIdx.x; rg < groups; rg += gridDim.x) {
-    const int64_t n = rg * BR_ROWS + slot;
-    const bool live = n < N;
-    const int64_t nr = live ? n : N - 1;
-    float y = 0.0f;
-    for (int64_t k0 = 0; k0 < K; k0 += BL_SLICE) {
-      const int cols = (int)(K - k0 < BL_SLICE ? K - k0 : (int64_t)BL_SLICE), jb0 = (int)(k0 / 128);
-      const int jend = jb0 + cols / 128;
-      int j = jb0 + part;
-      uint4 sw = make_uint4(0, 0, 0, 0), gw = sw;
-      float4 sc = make_float4(0, 0, 0, 0);
-      uint32_t rb = 0;
-      if (j < jend) {  // requested before the table is built, which does not need them
-        sw = __ldg(reinterpret_cast<const uint4 *>(sign + nr * ldw) + j);
-        gw = __ldg(reinterpret_cast<const uint4 *>(gmap + nr * ldw) + j);
-        sc = __ldg(reinterpret_cast<const float4 *>(bscale) + nr * nb + j);
-        rb = res[nr * nb + j];
-      }
-      __syncthreads();  // the previous slice's table is no longer read
-      for (int q = threadIdx.x; q < cols / 4; q += BR_THREADS) {
-        float x[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const __half_raw hr = {__ldg(X + k0 + 4 * q + i)};
-          bad |= (hr.x & 0x7C00u) == 0x7C00u;
-          x[i] = __half2float(__half(hr));
-        }
-        float v[16];
-        v[0] = 0.0f;
-#pragma unroll
-        for (int pt = 1; pt < 16; ++pt) {
-          // bits in ascending order: the highest set bit is added last
-          const int hi = 31 - __clz(pt);
-          v[pt] = (pt == (1 << hi)) ? x[hi] : v[pt ^ (1 << hi)] + x[hi];
-        }
-        float4 *dst = reinterpret_cast<float4 *>(lut + (q >> 5) * BL_BSTRIDE + (q & 31) * 16);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      }
-      __syncthreads();
-      for (int jl = threadIdx.x; jl < cols / 128; jl += BR_THREADS) {
-        float acc = 0.0f;
-        for (int t = 0; t < 32; ++t) acc += lut[jl * BL_BSTRIDE + t * 16 + 15];
-        xsum[jl] = acc;
-      }
-      __syncthreads();
-      for (; j < jend; j += BR_SPLIT) {
-        uint4 nsw = make_uint4(0, 0, 0, 0), ngw = nsw;
-        float4 nsc = make_float4(0, 0, 0, 0);
-        uint32_t nrb = 0;
-        if (j + BR_SPLIT < jend) {
-          nsw = __ldg(reinterpret_cast<const uint4 *>(sign + nr * ldw) + j + BR_SPLIT);
-          ngw = __ldg(reinterpret_cast<const uint4 *>(gmap + nr * ldw) + j + BR_SPLIT);
-          nsc = __ldg(reinterpret_cast<const float4 *>(bscale) + nr * nb + j + BR_SPLIT);
-          nrb = res[nr * nb + j + BR_SPLIT];
-        }
-        const float *lb = lut + (j - jb0) * BL_BSTRIDE;
-        const uint32_t swa[4] = {sw.x, sw.y, sw.z, sw.w};
-        // sum of x over the negative-sign columns: one lookup per nibble
-        float neg[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-#pragma unroll
-          for (int t = 0; t < 8; ++t) neg[q] += lb[(q * 8 + t) * 16 + ((swa[q] >> (4 * t)) & 15u)];
-        }
-        y = fmaf(sc.x, fmaf(-2.0f, (neg[0] + neg[1]) + (neg[2] + neg[3]), xsum[j - jb0]), y);
-        // sparse columns: (alpha_sp - alpha_c) * b * x
-        const float dsp = sc.y - sc.x;
-        const uint32_t gwa[4] = {gw.x, gw.y, gw.z, gw.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t g = gwa[q];
-          while (g) {
-            const int b = __ffs(g) - 1;
-            g &= g - 1;
-            const float xv = lb[(q * 8 + (b >> 2)) * 16 + (1 << (b & 3))];
-            y = fmaf(((swa[q] >> b) & 1u) ? -dsp : dsp, xv, y);
-          }
-        }
-        // salient columns: (alpha1 - alpha_c) * b1 + alpha2 * b2
-        const float d1 = sc.z - sc.x;
-        for (int i = 0; i < n_sal; ++i) {
-          const int c = ssal[j * n_sal + i];
-          const uint32_t wc = c < 64 ? (c < 32 ? sw.x : sw.y) : (c < 96 ? sw.z : sw.w);
-          const float cf = (((wc >> (c & 31)) & 1u) ? -d1 : d1) + (((rb >> i) & 1u) ? -sc.w : sc.w);
-          y = fmaf(cf, lb[(c >> 2) * 16 + (1 << (c & 3))], y);
-        }
-        sw = nsw;
-        gw = ngw;
-        sc = nsc;
-        rb = nrb;
-      }
-    }
-    y += __shfl_xor_sync(FULL, y, 1);
-    y += __shfl_xor_sync(FULL, y, 2);
-    if (live && part == 0) Y[n] = y;
-  }
-  if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
-}
-
-static cudaError_t launch_billm_gemv_lut(const uint16_t *X, const billm_weights *W, float *Y,
-                                         int32_t *d_status, cudaStream_t s) {
-  const size_t smem = (size_t)(BL_SLICE / 128) * (BL_BSTRIDE + 1) * 4 + (size_t)(W->K / 128) * W->n_sal;
-  static SmemOptIn opt_in;
-  if (cudaError_t e = opt_in(k_billm_gemv_lut, (int)smem)) return e;
-  int dev = 0, sms = 148, per_sm = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_billm_gemv_lut, BR_THREADS, smem) !=
-          cudaSuccess || per_sm < 1)
-    per_sm = 1;
-  const int64_t blocks =
-      std::min<int64_t>(ceil_div<int64_t>(W->N, BR_ROWS), (int64_t)sms * per_sm);
-  return launch_pdl(k_billm_gemv_lut, dim3((unsigned)blocks), dim3(BR_THREADS), smem, s, X, W->sign,
-                    W->gmap, W->res, W->sal, W->bscale, W->N, W->K, W->ldw_words, (int)W->n_sal, Y,
-                    d_status);
-}
-
 // Columns of K staged per pass: all of K when it fits, else a multiple of 512
 // (every thread then has blocks in each slice).
 static int br_slice(int mp, int64_t K) {
@@ -580,7 +467,7 @@ cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const b
     const cudaError_t e = launch_billm_gemm_tc(X, M, ldX, W, Y, ldY, d_status, s);
     if (e != cudaErrorNotSupported) return e;
   }
-  if (M == 1) return launch_billm_gemv_lut(X, W, Y, d_status, s);
+  if (M == 1) return launch_br_t<1>(X, M, ldX, W, Y, ldY, d_status, s);
   if (M == 2) return launch_br_t<2>(X, M, ldX, W, Y, ldY, d_status, s);
   if (M <= 4) return launch_br_t<4>(X, M, ldX, W, Y, ldY, d_status, s);
   if (M <= 8) return launch_br_t<8>(X, M, ldX, W, Y, ldY, d_status, s);

@@ -229,18 +229,31 @@ __device__ __forceinline__ void dc_compute(const DecodeBatch &p, uint8_t *smem, 
   __syncwarp();
   const int cnt = min(32, J.nchunks - 32 * cur.q);
   if (lane < DC_T) {
-    for (int cc = 0; cc < cnt; ++cc) {
+    // eight chunks at a time: their table loads are issued together
+    for (int c8 = 0; c8 < cnt; c8 += 8) {
+      int dv[8][MR];
+      float av[8];
 #pragma unroll
-      for (int m = 0; m < MR; ++m) f.gd[m] += fold_d[(m * 32 + cc) * (DC_T + 1) + lane];
-      if (--f.gleft == 0 || 32 * cur.q + cc + 1 == J.nchunks) {
-        const float al = fold_a[cc * (DC_T + 1) + lane];
+      for (int u = 0; u < 8; ++u) {
+        const int cc = min(c8 + u, 31);
 #pragma unroll
-        for (int m = 0; m < MR; ++m) {
-          f.acc[m] = fmaf(biased_int_to_float(f.gd[m] + INT_FLOAT_BIAS), al, f.acc[m]);
-          f.dt[m] += f.gd[m];
-          f.gd[m] = 0;
+        for (int m = 0; m < MR; ++m) dv[u][m] = fold_d[(m * 32 + cc) * (DC_T + 1) + lane];
+        av[u] = fold_a[cc * (DC_T + 1) + lane];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (c8 + u >= cnt) break;
+#pragma unroll
+        for (int m = 0; m < MR; ++m) f.gd[m] += dv[u][m];
+        if (--f.gleft == 0 || 32 * cur.q + c8 + u + 1 == J.nchunks) {
+#pragma unroll
+          for (int m = 0; m < MR; ++m) {
+            f.acc[m] = fmaf(biased_int_to_float(f.gd[m] + INT_FLOAT_BIAS), av[u], f.acc[m]);
+            f.dt[m] += f.gd[m];
+            f.gd[m] = 0;
+          }
+          f.gleft = J.gchunks;
         }
-        f.gleft = J.gchunks;
       }
     }
   }
@@ -267,9 +280,10 @@ __device__ __forceinline__ void dc_compute(const DecodeBatch &p, uint8_t *smem, 
 // the whole CTA is then one team of 256 threads per row: piece p (8 halves)
 // of a row belongs to thread p % 256, and 16 consecutive threads cover one
 // 128-element chunk.
+template <bool FUSED>
 __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *smem, int32_t *d_status) {
   __shared__ uint64_t red[QA_THREADS / 32];
-  if (!p.fused) {
+  if (!FUSED) {
     for (int j = 0; j < p.njobs; ++j) {
       const DecodeJob &J = p.job[j];
       uint4 *sA = reinterpret_cast<uint4 *>(smem + J.act_off);
@@ -378,7 +392,7 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
   if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
 }
 
-template <int MR>
+template <int MR, bool FUSED>
 __global__ void __launch_bounds__(DC_THREADS, 2)
 k_decode(const __grid_constant__ DecodeBatch p, int32_t *d_status) {
   extern __shared__ uint4 dc_smem4[];
@@ -399,23 +413,18 @@ k_decode(const __grid_constant__ DecodeBatch p, int32_t *d_status) {
 
   pdl_trigger();
   // with the weights known to be complete, the first banks are requested
-  // before waiting for the previous kernel in the stream
-  if (p.ready) {
-#pragma unroll
+  // before waiting for the previous kernel in the stream (its CTAs may still
+  // be running on this SM: one CTA per SM leaves room for the next kernel's)
+  for (int pass = 0; pass < 2; ++pass) {
+    if (pass == 1) pdl_wait();
+    if ((pass == 0) != (p.ready != 0)) continue;
+#pragma unroll 1
     for (int k = 0; k < DC_RING; ++k) {
       dc_issue(p, ld, dc_slot(ring, k, lane));
       if (ld.tile < p.ntiles) ld.advance(p, stride, lane);
     }
   }
-  pdl_wait();
-  if (!p.ready) {
-#pragma unroll
-    for (int k = 0; k < DC_RING; ++k) {
-      dc_issue(p, ld, dc_slot(ring, k, lane));
-      if (ld.tile < p.ntiles) ld.advance(p, stride, lane);
-    }
-  }
-  dc_setup_acts(p, smem, d_status);
+  dc_setup_acts<FUSED>(p, smem, d_status);
   __syncthreads();
 
   // the fold restarts at the first bank of every tile (slice 0, row 0)
@@ -443,10 +452,10 @@ bool decode_fits(int64_t M, int64_t K) {
          dc_act_bytes((int)M, (int)nchunks) <= DC_MAX_ACT_SMEM;
 }
 
-template <int MR>
+template <int MR, bool FUSED>
 static cudaError_t launch_decode_t(const DecodeBatch &p, size_t smem, int32_t *d_status,
                                    cudaStream_t s) {
-  auto kern = k_decode<MR>;
+  auto kern = k_decode<MR, FUSED>;
   static SmemOptIn opt_in;
   if (cudaError_t e = opt_in(kern, (int)smem)) return e;
   int dev = 0, sms = 148, per_sm = 1;
@@ -455,9 +464,12 @@ static cudaError_t launch_decode_t(const DecodeBatch &p, size_t smem, int32_t *d
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DC_THREADS, smem) != cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
-  // tiles go to CTAs first: with few tiles, one or two warps per CTA work and
-  // every SM streams
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(p.ntiles, (int64_t)per_sm * sms));
+  // One CTA per SM when the tiles do not fill two CTAs' warps on every SM:
+  // the SM then keeps room for a CTA of the next kernel in the stream, which
+  // starts its weight loads early. Long streams get two CTAs per SM (twice the
+  // loads in flight). Tiles go to CTAs first, so every SM streams.
+  const int64_t per = (p.ntiles > (int64_t)2 * sms * DC_WARPS && per_sm >= 2) ? 2 : 1;
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(p.ntiles, per * sms));
   return launch_pdl(kern, dim3((unsigned)blocks), dim3(DC_THREADS), smem, s, p, d_status);
 }
 
@@ -526,10 +538,14 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
   p.stage_pieces = (int)(stage / 16);
   const size_t smem = act + ring + std::max(fold, stage);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  if (MR <= 1) return launch_decode_t<1>(p, smem, d_status, s);
-  if (MR <= 2) return launch_decode_t<2>(p, smem, d_status, s);
-  if (MR <= 4) return launch_decode_t<4>(p, smem, d_status, s);
-  return launch_decode_t<8>(p, smem, d_status, s);
+#define BWTA_DC(R)                                                                              \
+  return fused ? launch_decode_t<R, true>(p, smem, d_status, s)                                 \
+               : launch_decode_t<R, false>(p, smem, d_status, s)
+  if (MR <= 1) BWTA_DC(1);
+  if (MR <= 2) BWTA_DC(2);
+  if (MR <= 4) BWTA_DC(4);
+  BWTA_DC(8);
+#undef BWTA_DC
 }
 
 int decode_max_jobs() { return DC_MAX_JOBS; }
