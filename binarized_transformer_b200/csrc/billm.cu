@@ -463,7 +463,10 @@ static cudaError_t launch_br_t(const uint16_t *X, int64_t M, int64_t ldX, const 
 cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,
                               float *Y, int64_t ldY, int32_t *d_status, cudaStream_t s) {
   if (M == 0 || W->N == 0) return cudaSuccess;
-  if (M >= 2) {  // tensor cores, when X satisfies the TMA alignment rules
+  // M <= 4 on CUDA cores (the weight rebuild of the tensor-core kernel costs
+  // as much at M = 2 as at M = 512); larger M on tensor cores, when X
+  // satisfies the TMA alignment rules.
+  if (M > 4) {
     const cudaError_t e = launch_billm_gemm_tc(X, M, ldX, W, Y, ldY, d_status, s);
     if (e != cudaErrorNotSupported) return e;
   }

@@ -13,38 +13,56 @@
 // -- the same fp32 operations, in the same order, as the tiled GEMM, so the
 // outputs agree bit for bit.
 //
-// Work is cut into tiles of DC_T = 8 weight rows of one projection, handed out
-// round-robin first across the CTAs, then across the warps of a CTA, so that
-// every SM streams even when there are few tiles. A warp walks its tiles in
-// slices of 32 chunks (128 elements = 4 words per plane) and banks of DC_P
-// rows: lane c copies chunk c of each row of a bank (512 contiguous bytes per
-// row and warp) and that chunk's weight scale into a per-warp shared-memory
-// ring with cp.async, DC_RING banks ahead of the bank it computes. Each lane
-// reads back only what it copied itself, so its own cp.async group wait is
-// the only synchronisation, and no register is held by a load in flight.
-// The integer dot of each (row, chunk) and the chunk's weight scale go to a
-// per-warp shared-memory table [chunk][row]; when a slice is complete, lane r
-// folds row r's chunks in order (sum a group's chunks, then one fma per
-// group), so the serial fp32 order costs a few instructions per chunk rather
-// than a shuffle per group.
+// Work is cut into tiles of DC_R = 16 weight rows of one projection; a CTA
+// takes tiles blockIdx.x, blockIdx.x + gridDim.x, ... (all of a tile's K at
+// once). Warp roles:
+//  * the copy warp (one thread) brings each tile into a ring of shared-memory
+//    stages with two bulk copies -- the tile's rows of sign words are one
+//    contiguous block (rows are ldw words apart), and so are its rows of
+//    weight scales -- completing on the stage's mbarrier; with the weights
+//    known to be complete it fills the ring before the kernel waits for the
+//    previous kernel in the stream;
+//  * eight dot warps compute the integer dots: warp w takes rows 2w and
+//    2w + 1 of the tile, lane c the 128-element chunks c, c + 32, ... (16
+//    contiguous bytes per lane, conflict-free), and write each chunk's dot
+//    (int16: |d| <= 128) and weight scale to a fold table [row][chunk] with an
+//    odd row pitch, then release the stage;
+//  * four fold warps take the tiles in turn (tile i: fold warp i mod 4):
+//    lane r walks row r's chunks in order (integer group sums, one fma per
+//    group) and writes Y -- reads at an odd pitch, so the 16 lanes hit 16
+//    banks. The fold is a serial chain per row; keeping it off the dot warps
+//    lets them run ahead by as many tiles as there are fold tables.
+// The activation planes of every job sit in shared memory for the whole
+// launch: copied (bit-plane input) or made in the kernel from the fp16 rows
+// with the exact integer threshold of quant.cuh.
+// Every mbarrier wait is bounded; on a timeout the CTA records
+// BWTA_STATUS_TIMEOUT, lets the copies it issued land and returns.
 #include <algorithm>
 
 #include "common.cuh"
 #include "quant.cuh"
+#include "tcgen05.cuh"
 #include "tma.cuh"
 
 namespace bwta {
 
-constexpr int DC_THREADS = 256, DC_WARPS = DC_THREADS / 32;
-constexpr int DC_T = 8;  // weight rows per tile
-constexpr int DC_P = 4;     // rows per bank
-constexpr int DC_RING = 4;  // banks in flight per warp
-static_assert(DC_T % DC_P == 0, "a bank never straddles a slice");
-constexpr int DC_SLOT_BYTES = DC_P * 32 * (16 + 4);  // bits + scales of one bank
+constexpr int DC_WARPS = 8;                      // dot warps
+constexpr int DC_CTHREADS = DC_WARPS * 32;       // dot threads (named barrier 1)
+constexpr int DC_FOLD_WARPS = 4;                 // fold warps
+constexpr int DC_COPY_WARP = DC_WARPS + DC_FOLD_WARPS;
+constexpr int DC_THREADS = (DC_COPY_WARP + 1) * 32;
+constexpr int DC_R = 16;                         // weight rows per tile
+constexpr int DC_RPW = DC_R / DC_WARPS;          // rows per dot warp
+constexpr int DC_MAX_STAGES = 16;
+constexpr int DC_MAX_TABS = 8;
 constexpr int DC_MAX_JOBS = 8;
-constexpr int DC_MAX_CHUNKS = 128;  // K <= 16384 (fused ternarization keeps a row in registers)
-constexpr size_t DC_MAX_ACT_SMEM = 48 * 1024;  // + rings (80 KB) + fold tables (<= 83 KB) <= 227 KB
-constexpr int DC_STAGE_BYTES = 24 * 1024;  // fused: fp16 rows staged per round (at least one row)
+constexpr int DC_MAX_CHUNKS = 128;               // K <= 16384
+constexpr size_t DC_MAX_ACT_SMEM = 48 * 1024;
+constexpr size_t DC_RING_BUDGET = 56 * 1024;     // bytes of weight tiles in flight per CTA
+constexpr size_t DC_TAB_BUDGET = 48 * 1024;      // fold tables (at least two)
+constexpr int DC_STAGE_ROWS_BYTES = 24 * 1024;   // fused: fp16 rows staged per round
+constexpr int DC_ROUND_ROWS = 32;                // fused: at most this many rows per round
+static_assert(DC_R == 16 && DC_RPW * DC_WARPS == DC_R, "fold lanes 0..15, two rows per warp");
 
 struct DecodeJob {
   const uint16_t *X;            // fused: fp16 rows [M][ldX]
@@ -60,7 +78,7 @@ struct DecodeJob {
   int32_t *dots;
   int64_t ldD;
   int64_t tile0;                // first global tile of this job
-  int M, nchunks, gchunks, nslices;
+  int M, nchunks, gchunks;
   int act_off;                  // byte offset of the job's planes in shared memory
   int vec;                      // X rows 16-byte aligned
 };
@@ -68,10 +86,21 @@ struct DecodeJob {
 struct DecodeBatch {
   DecodeJob job[DC_MAX_JOBS];
   int64_t ntiles;
-  int njobs, fused, ternary, ready;
-  int ring_off;                 // byte offset of the per-warp cp.async rings
-  int fold_off;                 // byte offset of the per-warp fold tables
-  int stage_off, stage_pieces;  // fused: fp16 staging area (16-byte pieces), over the fold tables
+  int njobs, ternary, ready;
+  int stages, stage_bits, stage_bytes;  // copy ring: depth, bytes of sign words / of a stage
+  int ring_off;
+  int ntabs, nfold;                     // fold tables (a multiple of nfold), active fold warps
+  int tab_off, tab_bytes, pitch;        // fold tables (pitch odd, in elements)
+  int stage_off, stage_pieces;          // fused: fp16 staging area (over the fold tables)
+  int red_off;                          // fused: per-row partial sums (over the fold tables)
+};
+
+struct DcBars {
+  uint64_t full[DC_MAX_STAGES];   // copy of the stage landed (transaction bytes)
+  uint64_t empty[DC_MAX_STAGES];  // the dot warps have read the stage (8 arrivals)
+  uint64_t tfull[DC_MAX_TABS];    // the fold table is written (8 arrivals)
+  uint64_t tempty[DC_MAX_TABS];   // the fold table is folded (1 arrival)
+  int32_t timeout;
 };
 
 // Shared-memory planes of one job: sA [M][nchunks] uint4 (mask), sS (sign),
@@ -88,35 +117,23 @@ __device__ __forceinline__ JobActs job_acts(uint8_t *smem, const DecodeJob &J) {
   return {a, s, p, reinterpret_cast<float *>(p + J.M * J.nchunks)};
 }
 
-// Position of a warp in its stream of (tile, slice, row) items.
-struct DcCursor {
-  int64_t tile, n0;
-  int j, q, r;
-  int c, g;  // this lane's chunk in the slice (32q + lane) and its weight group
+__device__ __forceinline__ int dc_job_of(const DecodeBatch &p, int64_t tile) {
+  int j = 0;
+  while (j + 1 < p.njobs && tile >= p.job[j + 1].tile0) ++j;
+  return j;
+}
 
-  __device__ void locate(const DecodeBatch &p, int lane) {
-    j = 0;
-    while (j + 1 < p.njobs && tile >= p.job[j + 1].tile0) ++j;
-    n0 = (tile - p.job[j].tile0) * DC_T;
-    set_chunk(p, lane);
-  }
-  __device__ void set_chunk(const DecodeBatch &p, int lane) {
-    c = 32 * q + lane;
-    g = c / p.job[j].gchunks;
-  }
-  __device__ void advance(const DecodeBatch &p, int64_t stride, int lane) {
-    r += DC_P;
-    if (r < DC_T) return;
-    r = 0;
-    if (++q < p.job[j].nslices) {
-      set_chunk(p, lane);
-      return;
-    }
-    q = 0;
-    tile += stride;
-    if (tile < p.ntiles) locate(p, lane);
-  }
-};
+// The dot warps' barrier (the fold and copy warps never take part).
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, %0;" ::"n"(DC_CTHREADS) : "memory"); }
+
+// Bulk copy global -> this CTA's shared memory (no multicast), completing on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
   // copies src_bytes (0..16) and fills the rest of the 16 bytes with zeros
@@ -124,165 +141,40 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t 
                "r"(src_bytes)
                : "memory");
 }
-__device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(dst)), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-// One ring slot: bits [DC_P][32 lanes] uint4, then scales [DC_P][32] fp32.
-struct DcSlot {
-  uint4 *bits;
-  float *alpha;
-};
-__device__ __forceinline__ DcSlot dc_slot(uint8_t *ring, int k, int lane) {
-  uint8_t *b = ring + k * DC_SLOT_BYTES;
-  return {reinterpret_cast<uint4 *>(b) + lane,
-          reinterpret_cast<float *>(b + DC_P * 32 * 16) + lane};
+// Bounded wait that also records a timeout for the whole CTA.
+__device__ __forceinline__ bool dc_wait(DcBars &b, uint64_t *bar, uint32_t parity) {
+  if (*(volatile int32_t *)&b.timeout) return false;
+  if (mbar_wait(bar, parity, 2000000000ull)) return true;
+  b.timeout = 1;
+  return false;
 }
 
-// Copy this lane's chunk of the bank at `cur` (rows r .. r + DC_P - 1) into
-// its ring slot and close one cp.async group (empty when there is no bank):
-// rows past N and chunks past K arrive as zeros.
-__device__ __forceinline__ void dc_issue(const DecodeBatch &p, const DcCursor &cur, DcSlot sl) {
-  if (cur.tile < p.ntiles) {
-    const DecodeJob &J = p.job[cur.j];
-    const bool cin = cur.c < J.nchunks;
+// ------------------------------------------------------------- activations
+// Warp sum of a uint64 (every lane gets the total).
+__device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
 #pragma unroll
-    for (int i = 0; i < DC_P; ++i) {
-      const int64_t n = cur.n0 + cur.r + i;
-      const bool in = cin && n < J.N;
-      cp_async16(sl.bits + i * 32, in ? J.wb + n * J.ldw + 4 * cur.c : J.wb, in ? 16u : 0u);
-      if (J.Y) cp_async4(sl.alpha + i * 32, in ? J.ws + n * J.G + cur.g : J.ws, in ? 4u : 0u);
-    }
-  }
-  cp_async_commit();
-}
-
-// Per-warp fold table: dots [MR][32 chunks][DC_T + 1] int, then scales
-// [32][DC_T + 1] fp32 (odd row stride: conflict-free by chunk and by row).
-template <int MR>
-__host__ __device__ constexpr int dc_fold_bytes() {
-  return (MR + 1) * 32 * (DC_T + 1) * 4;
-}
-
-// Running fold of the rows of the current tile (lane r < DC_T owns row r).
-template <int MR>
-struct DcFold {
-  float acc[MR];
-  int gd[MR], dt[MR];
-  int gleft;  // chunks left in the current weight group
-
-  __device__ void reset(int gchunks) {
-#pragma unroll
-    for (int m = 0; m < MR; ++m) {
-      acc[m] = 0.0f;
-      gd[m] = 0;
-      dt[m] = 0;
-    }
-    gleft = gchunks;
-  }
-};
-
-template <int MR>
-__device__ __forceinline__ void dc_compute(const DecodeBatch &p, uint8_t *smem, int *fold_d,
-                                           float *fold_a, const DcCursor &cur, DcSlot sl,
-                                           DcFold<MR> &f, int lane) {
-  const DecodeJob &J = p.job[cur.j];
-  const JobActs acts = job_acts(smem, J);
-  const bool cin = cur.c < J.nchunks;
-  uint4 w[DC_P];
-  float a[DC_P];
-#pragma unroll
-  for (int i = 0; i < DC_P; ++i) {
-    w[i] = sl.bits[i * 32];
-    a[i] = J.Y ? sl.alpha[i * 32] : 0.0f;
-  }
-  // integer dots of this bank's rows with every activation row
-#pragma unroll
-  for (int i = 0; i < DC_P; ++i) {
-    const int r = cur.r + i;
-#pragma unroll
-    for (int m = 0; m < MR; ++m) {
-      int d = 0;
-      if (cin && m < J.M) {
-        const uint4 A = acts.sA[m * J.nchunks + cur.c], S = acts.sS[m * J.nchunks + cur.c];
-        d = acts.sP[m * J.nchunks + cur.c] -
-            2 * popc4_csa(lop3_and_xor(A.x, S.x, w[i].x), lop3_and_xor(A.y, S.y, w[i].y),
-                          lop3_and_xor(A.z, S.z, w[i].z), lop3_and_xor(A.w, S.w, w[i].w));
-      }
-      fold_d[(m * 32 + lane) * (DC_T + 1) + r] = d;
-    }
-    fold_a[lane * (DC_T + 1) + r] = a[i];
-  }
-  if (cur.r + DC_P < DC_T) return;
-
-  // the slice is complete: lane r folds row r's chunks in order
-  __syncwarp();
-  const int cnt = min(32, J.nchunks - 32 * cur.q);
-  if (lane < DC_T) {
-    // eight chunks at a time: their table loads are issued together
-    for (int c8 = 0; c8 < cnt; c8 += 8) {
-      int dv[8][MR];
-      float av[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int cc = min(c8 + u, 31);
-#pragma unroll
-        for (int m = 0; m < MR; ++m) dv[u][m] = fold_d[(m * 32 + cc) * (DC_T + 1) + lane];
-        av[u] = fold_a[cc * (DC_T + 1) + lane];
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (c8 + u >= cnt) break;
-#pragma unroll
-        for (int m = 0; m < MR; ++m) f.gd[m] += dv[u][m];
-        if (--f.gleft == 0 || 32 * cur.q + c8 + u + 1 == J.nchunks) {
-#pragma unroll
-          for (int m = 0; m < MR; ++m) {
-            f.acc[m] = fmaf(biased_int_to_float(f.gd[m] + INT_FLOAT_BIAS), av[u], f.acc[m]);
-            f.dt[m] += f.gd[m];
-            f.gd[m] = 0;
-          }
-          f.gleft = J.gchunks;
-        }
-      }
-    }
-  }
-  __syncwarp();
-  if (cur.q + 1 < J.nslices) return;
-
-  // the tile is complete: row n0 + lane
-  const int64_t n = cur.n0 + lane;
-  if (lane < DC_T && n < J.N) {
-#pragma unroll
-    for (int m = 0; m < MR; ++m) {
-      if (m >= J.M) break;
-      if (J.Y) J.Y[m * J.ldY + n] = f.acc[m] * acts.ssc[m];
-      if (J.dots) J.dots[m * J.ldD + n] = f.dt[m];
-    }
-  }
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+  return v;
 }
 
 // Planes of every job into shared memory: copied (bit-plane input) or made
 // here from the fp16 rows with the exact integer threshold of quant.cuh (the
 // same planes and scales as bwta_quantize_pack_acts, bit for bit). For the
-// latter the rows are first copied into a staging area with cp.async -- as
-// many rows per round as fit, so that one memory latency covers them -- and
-// the whole CTA is then one team of 256 threads per row: piece p (8 halves)
-// of a row belongs to thread p % 256, and 16 consecutive threads cover one
-// 128-element chunk.
+// latter, rows are copied into a staging area with cp.async -- as many rows
+// per round as fit, so that one memory latency covers them -- and the 256
+// compute threads then make the planes of every staged row: pass 1 sums the
+// magnitudes of all the round's rows (one partial per row and warp), pass 2
+// derives each row's threshold from them and writes the row's bits and kept
+// sums, and the row scales follow -- four barriers per round. Piece q (8
+// halves) of a row belongs to thread q % 256; 16 consecutive threads cover
+// one 128-element chunk.
 template <bool FUSED>
 __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *smem, int32_t *d_status) {
-  __shared__ uint64_t red[QA_THREADS / 32];
+  const int tid = threadIdx.x, wid = tid / 32, lane = tid % 32;
   if (!FUSED) {
     for (int j = 0; j < p.njobs; ++j) {
       const DecodeJob &J = p.job[j];
@@ -291,31 +183,35 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
       int *sP = reinterpret_cast<int *>(sS + J.M * J.nchunks);
       float *ssc = reinterpret_cast<float *>(sP + J.M * J.nchunks);
       const int nch = J.nchunks;
-      for (int idx = threadIdx.x; idx < J.M * nch; idx += DC_THREADS) {
+      for (int idx = tid; idx < J.M * nch; idx += DC_CTHREADS) {
         const int m = idx / nch, c = idx % nch;
         const uint4 v = __ldg(reinterpret_cast<const uint4 *>(J.am + m * J.lda) + c);
         sA[idx] = v;
         sS[idx] = __ldg(reinterpret_cast<const uint4 *>(J.as + m * J.lda) + c);
         sP[idx] = __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
       }
-      for (int m = threadIdx.x; m < J.M; m += DC_THREADS) ssc[m] = J.ascale ? __ldg(J.ascale + m) : 0.0f;
+      for (int m = tid; m < J.M; m += DC_CTHREADS) ssc[m] = J.ascale ? __ldg(J.ascale + m) : 0.0f;
     }
+    cbar();
     return;
   }
   uint4 *stage = reinterpret_cast<uint4 *>(smem + p.stage_off);
+  uint64_t *red_s = reinterpret_cast<uint64_t *>(smem + p.red_off);  // [row][warp]
+  uint64_t *red_k = red_s + DC_ROUND_ROWS * DC_WARPS;
+  uint64_t *red_n = red_k + DC_ROUND_ROWS * DC_WARPS;
   bool bad = false;
   int j = 0, m = 0;  // next row to stage
   while (j < p.njobs) {
     // one round: stage rows (j, m) ... while they fit
     const int j0 = j, m0 = m;
-    int used = 0;  // pieces of 16 bytes
-    while (j < p.njobs) {
+    int used = 0, nr = 0;  // pieces of 16 bytes, rows
+    while (j < p.njobs && nr < DC_ROUND_ROWS) {
       const DecodeJob &J = p.job[j];
       const int pieces = J.nchunks * 16;
       if (used > 0 && used + pieces > p.stage_pieces) break;
       const uint16_t *xr = J.X + m * J.ldX;
       const int64_t K = J.K;
-      for (int q = threadIdx.x; q < pieces; q += DC_THREADS) {
+      for (int q = tid; q < pieces; q += DC_CTHREADS) {
         const int64_t k0 = (int64_t)q * 8;
         uint4 *dst = stage + used + q;
         if (k0 >= K) {
@@ -327,118 +223,316 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
         }
       }
       used += pieces;
+      ++nr;
       if (++m == J.M) {
         m = 0;
         ++j;
       }
     }
     cp_async_wait_all();
-    __syncthreads();
-    // ternarize the staged rows
-    int off = 0;
-    for (int jj = j0, mm = m0; off < used;) {
-      const DecodeJob &J = p.job[jj];
-      const int nch = J.nchunks, steps = (nch + 15) / 16;
-      const int64_t K = J.K;
-      uint4 *sA = reinterpret_cast<uint4 *>(smem + J.act_off);
-      uint4 *sS = sA + J.M * nch;
-      float *ssc = reinterpret_cast<float *>(reinterpret_cast<int *>(sS + J.M * nch) + J.M * nch);
-      uint32_t *mrow = reinterpret_cast<uint32_t *>(sA + mm * nch);
-      uint32_t *srow = reinterpret_cast<uint32_t *>(sS + mm * nch);
-      const uint4 *row = stage + off;
-      uint64_t S = 0;
-      for (int st = 0; st < steps; ++st) {
-        const int q = st * DC_THREADS + threadIdx.x;
-        if (q < nch * 16) S += sum_mag8(row[q], bad);
-      }
-      S = team_sum_u64<QA_THREADS>(S, red);
-      const uint32_t hT = p.ternary ? mag_threshold_pattern(S / (uint64_t)(2 * K)) : 0u;
-      uint64_t ks = 0, kn = 0;
-      for (int st = 0; st < steps; ++st) {  // uniform trip count: store_chunk shuffles
-        const int q = st * DC_THREADS + threadIdx.x, chunk = q / 16;
-        const uint4 v = q < nch * 16 ? row[q] : make_uint4(0, 0, 0, 0);
-        const int64_t k0 = (int64_t)q * 8;
-        uint32_t kb, sb;
-        if (p.ternary) keep8<true>(v, hT, k0, K, kb, sb, ks);
-        else keep8<false>(v, hT, k0, K, kb, sb, ks);
-        kn += __popc(kb);
-        store_chunk(kb, sb, mrow, srow, chunk, chunk < nch);
-      }
-      if (p.ternary) {
-        ks = team_sum_u64<QA_THREADS>(ks, red);
-        kn = team_sum_u64<QA_THREADS>(kn, red);
-        if (threadIdx.x == 0) ssc[mm] = row_scale(ks, kn);
-      } else if (threadIdx.x == 0) {
-        ssc[mm] = row_scale(S, (uint64_t)K);
-      }
-      off += nch * 16;
-      if (++mm == J.M) {
-        mm = 0;
-        ++jj;
+    cbar();
+    // pass 1: magnitude sums of every staged row
+    {
+      int off = 0;
+      for (int r = 0, jj = j0, mm = m0; r < nr; ++r) {
+        const DecodeJob &J = p.job[jj];
+        const int pieces = J.nchunks * 16;
+        const uint4 *row = stage + off;
+        uint64_t S = 0;
+        for (int q = tid; q < pieces; q += DC_CTHREADS) S += sum_mag8(row[q], bad);
+        S = warp_sum_u64(S);
+        if (lane == 0) red_s[r * DC_WARPS + wid] = S;
+        off += pieces;
+        if (++mm == J.M) {
+          mm = 0;
+          ++jj;
+        }
       }
     }
-    __syncthreads();  // the staging area is free again; the planes are written
+    cbar();
+    // pass 2: threshold, bit planes, kept sums
+    {
+      int off = 0;
+      for (int r = 0, jj = j0, mm = m0; r < nr; ++r) {
+        const DecodeJob &J = p.job[jj];
+        const int nch = J.nchunks, pieces = nch * 16;
+        const int steps = (pieces + DC_CTHREADS - 1) / DC_CTHREADS;
+        const int64_t K = J.K;
+        uint64_t S = 0;
+#pragma unroll
+        for (int w = 0; w < DC_WARPS; ++w) S += red_s[r * DC_WARPS + w];
+        const uint32_t hT = p.ternary ? mag_threshold_pattern(S / (uint64_t)(2 * K)) : 0u;
+        uint4 *sA = reinterpret_cast<uint4 *>(smem + J.act_off);
+        uint32_t *mrow = reinterpret_cast<uint32_t *>(sA + mm * nch);
+        uint32_t *srow = reinterpret_cast<uint32_t *>(sA + J.M * nch + mm * nch);
+        const uint4 *row = stage + off;
+        uint64_t ks = 0, kn = 0;
+        for (int st = 0; st < steps; ++st) {  // uniform trip count: store_chunk shuffles
+          const int q = st * DC_CTHREADS + tid, chunk = q / 16;
+          const uint4 v = q < pieces ? row[q] : make_uint4(0, 0, 0, 0);
+          const int64_t k0 = (int64_t)q * 8;
+          uint32_t kb, sb;
+          if (p.ternary) keep8<true>(v, hT, k0, K, kb, sb, ks);
+          else keep8<false>(v, hT, k0, K, kb, sb, ks);
+          kn += __popc(kb);
+          store_chunk(kb, sb, mrow, srow, chunk, chunk < nch);
+        }
+        ks = warp_sum_u64(ks);
+        kn = warp_sum_u64(kn);
+        if (lane == 0) {
+          red_k[r * DC_WARPS + wid] = ks;
+          red_n[r * DC_WARPS + wid] = kn;
+        }
+        off += pieces;
+        if (++mm == J.M) {
+          mm = 0;
+          ++jj;
+        }
+      }
+    }
+    cbar();
+    // row scales (one thread per staged row)
+    if (tid < nr) {
+      int jj = j0, mm = m0;
+      for (int r = 0; r < tid; ++r)
+        if (++mm == p.job[jj].M) {
+          mm = 0;
+          ++jj;
+        }
+      const DecodeJob &J = p.job[jj];
+      float *ssc = reinterpret_cast<float *>(smem + J.act_off + (size_t)J.M * J.nchunks * 36);
+      uint64_t a = 0, b = 0;
+      if (p.ternary) {
+#pragma unroll
+        for (int w = 0; w < DC_WARPS; ++w) {
+          a += red_k[tid * DC_WARPS + w];
+          b += red_n[tid * DC_WARPS + w];
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < DC_WARPS; ++w) a += red_s[tid * DC_WARPS + w];
+        b = (uint64_t)J.K;
+      }
+      ssc[mm] = row_scale(a, b);
+    }
+    cbar();  // the staging area and the partial sums are free again
   }
   // popcounts of the mask chunks
   for (int jj = 0; jj < p.njobs; ++jj) {
     const DecodeJob &J = p.job[jj];
     const uint4 *sA = reinterpret_cast<const uint4 *>(smem + J.act_off);
     int *sP = reinterpret_cast<int *>(const_cast<uint4 *>(sA) + 2 * J.M * J.nchunks);
-    for (int idx = threadIdx.x; idx < J.M * J.nchunks; idx += DC_THREADS) {
+    for (int idx = tid; idx < J.M * J.nchunks; idx += DC_CTHREADS) {
       const uint4 v = sA[idx];
       sP[idx] = __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
     }
   }
   if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
+  cbar();
+}
+
+// ------------------------------------------------------------------ kernel
+// Fold table b: d [MR][DC_R][pitch] int16, then alpha [DC_R][pitch] fp32.
+__host__ __device__ __forceinline__ size_t dc_tab_d_bytes(int mr, int pitch) {
+  return ((size_t)mr * DC_R * pitch * 2 + 15) / 16 * 16;
 }
 
 template <int MR, bool FUSED>
-__global__ void __launch_bounds__(DC_THREADS, 2)
+__global__ void __launch_bounds__(DC_THREADS, 1)
 k_decode(const __grid_constant__ DecodeBatch p, int32_t *d_status) {
   extern __shared__ uint4 dc_smem4[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(dc_smem4);
+  __shared__ DcBars bars;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  int *fold_d = reinterpret_cast<int *>(smem + p.fold_off + warp * dc_fold_bytes<MR>());
-  float *fold_a = reinterpret_cast<float *>(fold_d + MR * 32 * (DC_T + 1));
-  uint8_t *ring = smem + p.ring_off + warp * (DC_RING * DC_SLOT_BYTES);
-  // tiles go round-robin over the CTAs first, then over the warps of a CTA
-  const int64_t stride = (int64_t)gridDim.x * DC_WARPS;
+  const int64_t stride = gridDim.x;
+  uint8_t *ring = smem + p.ring_off;
 
-  DcCursor ld, cur;  // the bank being copied, the bank being computed
-  ld.tile = (int64_t)warp * gridDim.x + blockIdx.x;
-  ld.q = 0;
-  ld.r = 0;
-  if (ld.tile < p.ntiles) ld.locate(p, lane);
-  cur = ld;
-
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], DC_WARPS);
+    }
+    for (int t = 0; t < p.ntabs; ++t) {
+      mbar_init(&bars.tfull[t], DC_WARPS);
+      mbar_init(&bars.tempty[t], 1);
+    }
+    bars.timeout = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
   pdl_trigger();
-  // with the weights known to be complete, the first banks are requested
-  // before waiting for the previous kernel in the stream (its CTAs may still
-  // be running on this SM: one CTA per SM leaves room for the next kernel's)
-  for (int pass = 0; pass < 2; ++pass) {
-    if (pass == 1) pdl_wait();
-    if ((pass == 0) != (p.ready != 0)) continue;
-#pragma unroll 1
-    for (int k = 0; k < DC_RING; ++k) {
-      dc_issue(p, ld, dc_slot(ring, k, lane));
-      if (ld.tile < p.ntiles) ld.advance(p, stride, lane);
+
+  if (warp == DC_COPY_WARP) {
+    // ------------------------------------------------ copy warp
+    if (lane == 0) {
+      if (!p.ready) pdl_wait();  // weights may still be written by the previous kernel
+      int i = 0;
+      for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += stride, ++i) {
+        const int s = i % p.stages;
+        if (i >= p.stages && !dc_wait(bars, &bars.empty[s], ((i / p.stages) - 1) & 1)) break;
+        const DecodeJob &J = p.job[dc_job_of(p, tile)];
+        const int64_t n0 = (tile - J.tile0) * DC_R;
+        const int64_t rows = J.N - n0 < DC_R ? J.N - n0 : DC_R;
+        uint8_t *st = ring + (size_t)s * p.stage_bytes;
+        const uint32_t bbytes = (uint32_t)(rows * J.ldw * 4);
+        const uint32_t sbytes = J.Y ? (uint32_t)(rows * J.G * 4) : 0u, s16 = sbytes & ~15u;
+        // a scale tail that is not a whole 16 bytes: plain loads (published by the arrive)
+        float *sdst = reinterpret_cast<float *>(st + p.stage_bits);
+        for (uint32_t q = s16 / 4; q < sbytes / 4; ++q) sdst[q] = __ldg(J.ws + n0 * J.G + q);
+        mbar_arrive_expect_tx(&bars.full[s], bbytes + s16);
+        bulk_load(st, J.wb + n0 * J.ldw, bbytes, &bars.full[s]);
+        if (s16) bulk_load(sdst, J.ws + n0 * J.G, s16, &bars.full[s]);
+      }
+      // Copies still in flight (after a timeout) land before the CTA exits; a
+      // stage is refilled only after its previous copy was consumed, so only
+      // the last `stages` copies can be pending.
+      bool drained = true;
+      for (int q = i > p.stages ? i - p.stages : 0; q < i; ++q)
+        drained &= mbar_wait(&bars.full[q % p.stages], (q / p.stages) & 1, DRAIN_NS);
+      if (!drained) flag_status(d_status, BWTA_STATUS_DRAIN);
+    }
+    return;
+  }
+
+  if (warp >= DC_WARPS) {
+    // ------------------------------------------------ fold warps
+    pdl_wait();  // outputs follow the previous kernel in the stream
+    // Fold warp f takes tiles f, f + nfold, ...; with ntabs a multiple of
+    // nfold, table b = i % ntabs is only ever folded by warp b % nfold, so
+    // each table's barriers are waited on in order by one warp (a parity
+    // wait never sees a phase two ahead).
+    const int f = warp - DC_WARPS;
+    int i = f;
+    for (int64_t tile = blockIdx.x + (int64_t)f * stride; f < p.nfold && tile < p.ntiles;
+         tile += (int64_t)p.nfold * stride, i += p.nfold) {
+      const int b = i % p.ntabs;
+      if (!__all_sync(FULL, dc_wait(bars, &bars.tfull[b], (i / p.ntabs) & 1))) break;
+      const DecodeJob &J = p.job[dc_job_of(p, tile)];
+      const JobActs acts = job_acts(smem, J);
+      const uint8_t *tab = smem + p.tab_off + (size_t)b * p.tab_bytes;
+      const int nch = J.nchunks, gc = J.gchunks;
+      const int64_t n = (tile - J.tile0) * DC_R + lane;
+      if (lane < DC_R) {
+        // lane r walks row r's chunks in order
+        const int16_t *dr = reinterpret_cast<const int16_t *>(tab) + lane * p.pitch;
+        const float *ar = reinterpret_cast<const float *>(tab + dc_tab_d_bytes(MR, p.pitch)) + lane * p.pitch;
+        const int dstride = DC_R * p.pitch;
+        float acc[MR];
+        int dt[MR], gd[MR];
+#pragma unroll
+        for (int m = 0; m < MR; ++m) {
+          acc[m] = 0.0f;
+          dt[m] = 0;
+          gd[m] = 0;
+        }
+        if (gc == 1) {  // one weight group per chunk (group 128): every chunk closes a group
+          constexpr int U = MR <= 2 ? 16 : 4;  // chunks whose loads are issued together
+          int c = 0;
+          for (; c + U <= nch; c += U) {
+            float av[U], dv[U][MR];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              av[u] = ar[c + u];
+#pragma unroll
+              for (int m = 0; m < MR; ++m) {
+                const int d = dr[m * dstride + c + u];
+                dt[m] += d;
+                dv[u][m] = biased_int_to_float(d + INT_FLOAT_BIAS);
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+              for (int m = 0; m < MR; ++m) acc[m] = fmaf(dv[u][m], av[u], acc[m]);
+          }
+          for (; c < nch; ++c) {
+            const float a = ar[c];
+#pragma unroll
+            for (int m = 0; m < MR; ++m) {
+              const int d = dr[m * dstride + c];
+              acc[m] = fmaf(biased_int_to_float(d + INT_FLOAT_BIAS), a, acc[m]);
+              dt[m] += d;
+            }
+          }
+        } else {
+          int left = gc;
+          for (int c = 0; c < nch; ++c) {
+#pragma unroll
+            for (int m = 0; m < MR; ++m) gd[m] += dr[m * dstride + c];
+            if (--left == 0 || c + 1 == nch) {
+              const float a = ar[c];
+#pragma unroll
+              for (int m = 0; m < MR; ++m) {
+                acc[m] = fmaf(biased_int_to_float(gd[m] + INT_FLOAT_BIAS), a, acc[m]);
+                dt[m] += gd[m];
+                gd[m] = 0;
+              }
+              left = gc;
+            }
+          }
+        }
+        if (n < J.N) {
+#pragma unroll
+          for (int m = 0; m < MR; ++m) {
+            if (m >= J.M) break;
+            if (J.Y) J.Y[m * J.ldY + n] = acc[m] * acts.ssc[m];
+            if (J.dots) J.dots[m * J.ldD + n] = dt[m];
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.tempty[b]);
+    }
+    return;
+  }
+
+  // ------------------------------------------------ dot warps
+  pdl_wait();  // activations follow the previous kernel in the stream
+  dc_setup_acts<FUSED>(p, smem, d_status);
+
+  int i = 0;
+  for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += stride, ++i) {
+    const int s = i % p.stages, b = i % p.ntabs;
+    const DecodeJob &J = p.job[dc_job_of(p, tile)];
+    bool ok = dc_wait(bars, &bars.full[s], (i / p.stages) & 1);
+    if (ok && i >= p.ntabs) ok = dc_wait(bars, &bars.tempty[b], ((i / p.ntabs) - 1) & 1);
+    if (!__all_sync(FULL, ok)) break;  // warp-uniform: the loop below synchronizes the warp
+    const JobActs acts = job_acts(smem, J);
+    const uint8_t *st = ring + (size_t)s * p.stage_bytes;
+    uint8_t *tab = smem + p.tab_off + (size_t)b * p.tab_bytes;
+    int16_t *td = reinterpret_cast<int16_t *>(tab);
+    float *ta = reinterpret_cast<float *>(tab + dc_tab_d_bytes(MR, p.pitch));
+    const int nch = J.nchunks, gc = J.gchunks;
+    // integer dots of this warp's rows with every activation row
+#pragma unroll
+    for (int rr = 0; rr < DC_RPW; ++rr) {
+      const int r = warp * DC_RPW + rr;
+      const uint4 *bits = reinterpret_cast<const uint4 *>(st + (size_t)r * J.ldw * 4);
+      const float *sc = reinterpret_cast<const float *>(st + p.stage_bits) + r * J.G;
+      for (int c = lane; c < nch; c += 32) {
+        const uint4 w = bits[c];
+        ta[r * p.pitch + c] = J.Y ? sc[gc == 1 ? c : c / gc] : 0.0f;
+#pragma unroll
+        for (int m = 0; m < MR; ++m) {
+          int d = 0;
+          if (m < J.M) {
+            const uint4 A = acts.sA[m * nch + c], S = acts.sS[m * nch + c];
+            d = acts.sP[m * nch + c] -
+                2 * popc4_csa(lop3_and_xor(A.x, S.x, w.x), lop3_and_xor(A.y, S.y, w.y),
+                              lop3_and_xor(A.z, S.z, w.z), lop3_and_xor(A.w, S.w, w.w));
+          }
+          td[(m * DC_R + r) * p.pitch + c] = (int16_t)d;
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&bars.empty[s]);
+      mbar_arrive(&bars.tfull[b]);
     }
   }
-  dc_setup_acts<FUSED>(p, smem, d_status);
-  __syncthreads();
-
-  // the fold restarts at the first bank of every tile (slice 0, row 0)
-  DcFold<MR> f;
-  for (int k = 0; cur.tile < p.ntiles; k = (k + 1 == DC_RING) ? 0 : k + 1) {
-    if (cur.q == 0 && cur.r == 0) f.reset(p.job[cur.j].gchunks);
-    cp_async_wait<DC_RING - 1>();  // this lane's copies of bank `cur` have landed
-    const DcSlot sl = dc_slot(ring, k, lane);
-    dc_compute<MR>(p, smem, fold_d, fold_a, cur, sl, f, lane);
-    dc_issue(p, ld, sl);           // the slot is free again: the bank DC_RING ahead
-    if (ld.tile < p.ntiles) ld.advance(p, stride, lane);
-    cur.advance(p, stride, lane);
-  }
-  cp_async_wait<0>();
+  if (lane == 0 && warp == 0 && *(volatile int32_t *)&bars.timeout)
+    flag_status(d_status, BWTA_STATUS_TIMEOUT);
 }
 
 // ------------------------------------------------------------------ host
@@ -458,25 +552,21 @@ static cudaError_t launch_decode_t(const DecodeBatch &p, size_t smem, int32_t *d
   auto kern = k_decode<MR, FUSED>;
   static SmemOptIn opt_in;
   if (cudaError_t e = opt_in(kern, (int)smem)) return e;
-  int dev = 0, sms = 148, per_sm = 1;
+  int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DC_THREADS, smem) != cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
-  // One CTA per SM when the tiles do not fill two CTAs' warps on every SM:
-  // the SM then keeps room for a CTA of the next kernel in the stream, which
-  // starts its weight loads early. Long streams get two CTAs per SM (twice the
-  // loads in flight). Tiles go to CTAs first, so every SM streams.
-  const int64_t per = (p.ntiles > (int64_t)2 * sms * DC_WARPS && per_sm >= 2) ? 2 : 1;
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(p.ntiles, per * sms));
+  // One CTA per SM (tiles go to CTAs round-robin, so every SM streams); an
+  // SM keeps room for a CTA of the next kernel in the stream, which fills its
+  // own ring while this one finishes.
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(p.ntiles, sms));
   return launch_pdl(kern, dim3((unsigned)blocks), dim3(DC_THREADS), smem, s, p, d_status);
 }
 
 cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mode, bool ready,
                           int32_t *d_status, cudaStream_t s) {
   DecodeBatch p = {};
-  int MR = 1;
+  int MR = 1, nch_max = 1;
+  int64_t ldw_max = 4, G_max = 1;
   size_t act = 0;
   int nj = 0;
   for (int i = 0; i < njobs; ++i) {
@@ -502,48 +592,61 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
     J.nchunks = (int)ceil_div<int64_t>(ceil_div<int64_t>(in.K, 32), 4);
     J.gchunks = in.group ? (int)(in.group / 128) : J.nchunks;
     J.G = in.group ? ceil_div<int64_t>(in.K, in.group) : 1;
-    J.nslices = ceil_div(J.nchunks, 32);
     J.vec = (reinterpret_cast<uintptr_t>(in.X) & 15u) == 0 && in.ldX % 8 == 0;
     J.act_off = (int)act;
     act += dc_act_bytes(J.M, J.nchunks);
     J.tile0 = p.ntiles;
-    p.ntiles += ceil_div<int64_t>(in.N, DC_T);
+    p.ntiles += ceil_div<int64_t>(in.N, DC_R);
     MR = std::max(MR, J.M);
+    nch_max = std::max(nch_max, J.nchunks);
+    ldw_max = std::max(ldw_max, J.ldw);
+    G_max = std::max(G_max, J.G);
     ++nj;
   }
   if (nj == 0) return cudaSuccess;
   if (act > DC_MAX_ACT_SMEM) return cudaErrorInvalidValue;
   p.njobs = nj;
-  p.fused = fused;
   p.ternary = mode == BWTA_TERNARY;
   p.ready = ready;
+  const int mr = MR <= 1 ? 1 : MR <= 2 ? 2 : MR <= 4 ? 4 : 8;
+  // copy ring: DC_R rows of sign words and of scales of the widest job
+  p.stage_bits = (int)(DC_R * ldw_max * 4);
+  p.stage_bytes = (int)((p.stage_bits + DC_R * G_max * 4 + 15) / 16 * 16);
+  p.stages = (int)std::min<size_t>(DC_MAX_STAGES,
+                                   std::max<size_t>(2, DC_RING_BUDGET / (size_t)p.stage_bytes));
   p.ring_off = (int)act;
-  const size_t ring = (size_t)DC_WARPS * DC_RING * DC_SLOT_BYTES;
-  p.fold_off = (int)(act + ring);
-  const size_t fold = (size_t)DC_WARPS * (MR <= 1 ? dc_fold_bytes<1>() : MR <= 2 ? dc_fold_bytes<2>()
-                                          : MR <= 4 ? dc_fold_bytes<4>() : dc_fold_bytes<8>());
-  size_t stage = 0;
-  if (fused) {  // every staged row fits; as many rows per round as DC_STAGE_BYTES holds
+  const size_t ring = (size_t)p.stages * p.stage_bytes;
+  // fold tables, then (fused) the staging area and partial sums over them
+  p.pitch = nch_max | 1;
+  p.tab_bytes = (int)((dc_tab_d_bytes(mr, p.pitch) + (size_t)DC_R * p.pitch * 4 + 15) / 16 * 16);
+  p.tab_off = (int)(act + ring);
+  size_t over = 0;
+  if (fused) {  // every staged row fits; as many rows per round as the staging area holds
     size_t rows_bytes = 0, row_max = 0;
     for (int i = 0; i < nj; ++i) {
       const size_t rb = (size_t)p.job[i].nchunks * 256;
       rows_bytes += rb * p.job[i].M;
       row_max = std::max(row_max, rb);
     }
-    stage = std::max(row_max, std::min(rows_bytes, (size_t)DC_STAGE_BYTES));
+    const size_t stage = std::max(row_max, std::min(rows_bytes, (size_t)DC_STAGE_ROWS_BYTES));
+    p.stage_off = p.tab_off;
+    p.stage_pieces = (int)(stage / 16);
+    p.red_off = (int)(p.tab_off + stage);
+    over = stage + (size_t)3 * DC_ROUND_ROWS * DC_WARPS * 8;
   }
-  // the staging area is used only before the main loop: it shares the space
-  // of the fold tables (not of the rings, whose first copies are in flight)
-  p.stage_off = p.fold_off;
-  p.stage_pieces = (int)(stage / 16);
-  const size_t smem = act + ring + std::max(fold, stage);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  const size_t limit = 227 * 1024;
+  p.ntabs = (int)std::max<size_t>(2, std::min<size_t>(DC_MAX_TABS, DC_TAB_BUDGET / p.tab_bytes));
+  while (p.ntabs > 2 && act + ring + std::max((size_t)p.ntabs * p.tab_bytes, over) > limit) --p.ntabs;
+  p.nfold = std::min(p.ntabs, DC_FOLD_WARPS);
+  p.ntabs -= p.ntabs % p.nfold;
+  const size_t smem = act + ring + std::max((size_t)p.ntabs * p.tab_bytes, over);
+  if (smem > limit) return cudaErrorInvalidValue;
 #define BWTA_DC(R)                                                                              \
   return fused ? launch_decode_t<R, true>(p, smem, d_status, s)                                 \
                : launch_decode_t<R, false>(p, smem, d_status, s)
-  if (MR <= 1) BWTA_DC(1);
-  if (MR <= 2) BWTA_DC(2);
-  if (MR <= 4) BWTA_DC(4);
+  if (mr == 1) BWTA_DC(1);
+  if (mr == 2) BWTA_DC(2);
+  if (mr == 4) BWTA_DC(4);
   BWTA_DC(8);
 #undef BWTA_DC
 }

@@ -53,48 +53,101 @@ __device__ __forceinline__ uint4 load_half8(const uint16_t *row, int64_t k0, int
 // is a multiple of 2^-24 below 2^16, so a sum of 8 needs at most 19 + 24 = 43
 // significant bits: its fp64 sum is exact in any order, and so is its product
 // with 2^24 and the conversion to an integer (the same value as the sum of
-// mag_units of the 8 patterns, for one conversion and one add per element).
-__device__ __forceinline__ double half_mag(uint32_t hm) {
-  return (double)__half2float(__ushort_as_half((unsigned short)hm));
-}
+// mag_units of the 8 patterns).
 __device__ __forceinline__ uint64_t units_of(double d) { return (uint64_t)(d * 16777216.0); }
 
-__device__ __forceinline__ uint64_t sum_mag8(const uint4 &v, bool &bad) {
+// Both halves of a word as fp64 (exact): one conversion per element.
+__device__ __forceinline__ void f16x2_to_f64(uint32_t w, double &lo, double &hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f64.f16 %0, l;\n\tcvt.f64.f16 %1, h;\n\t}"
+      : "=d"(lo), "=d"(hi)
+      : "r"(w));
+}
+// Sum of the 8 halves of four words of magnitude patterns (sign bits clear),
+// in a balanced tree. A non-finite pattern makes the sum non-finite.
+__device__ __forceinline__ double f64_sum8(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  double a0, a1, b0, b1, c0, c1, d0, d1;
+  f16x2_to_f64(a, a0, a1);
+  f16x2_to_f64(b, b0, b1);
+  f16x2_to_f64(c, c0, c1);
+  f16x2_to_f64(d, d0, d1);
+  return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+}
+__device__ __forceinline__ bool finite_f64(double d) { return fabs(d) < __longlong_as_double(0x7FF0000000000000ll); }
+
+constexpr uint32_t MAG2 = 0x7FFF7FFFu;  // the magnitude bits of two halves
+
+// The same sum one element at a time, leaving out (and reporting) the
+// non-finite ones; taken only when the fast sum is not finite.
+__device__ __forceinline__ uint64_t sum_mag8_nonfinite(uint4 v, bool &bad) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  double d = 0.0;
+  uint32_t f[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t hm = (w[i >> 1] >> (16 * (i & 1))) & 0x7FFFu;
-    bad |= hm >= 0x7C00u;
-    d += half_mag(hm < 0x7C00u ? hm : 0u);
+  for (int j = 0; j < 4; ++j) {
+    uint32_t r = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t hm = (w[j] >> (16 * h)) & 0x7FFFu;
+      bad |= hm >= 0x7C00u;
+      r |= (hm < 0x7C00u ? hm : 0u) << (16 * h);
+    }
+    f[j] = r;
   }
-  return units_of(d);
+  return units_of(f64_sum8(f[0], f[1], f[2], f[3]));
+}
+
+__device__ __forceinline__ uint64_t sum_mag8(const uint4 &v, bool &bad) {
+  const double d = f64_sum8(v.x & MAG2, v.y & MAG2, v.z & MAG2, v.w & MAG2);
+  if (finite_f64(d)) return units_of(d);
+  return sum_mag8_nonfinite(v, bad);
+}
+
+// Bit i of the result = bit 15 + 16*(i&1) of word i>>1, for 8 halves held in
+// four words whose other bits are clear.
+__device__ __forceinline__ uint32_t gather_bit15(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  const uint32_t t = (a >> 15) | (b >> 13) | (c >> 11) | (d >> 9);  // bits 2j and 2j + 16
+  return (t | (t >> 15)) & 0xFFu;
 }
 
 // keep / sign bit patterns of 8 halves, plus the sum of the kept magnitudes.
+// Ternary: keep iff the magnitude pattern exceeds hT, two halves per integer
+// subtract: per half, (0x8000 | hT) - hm has bit 15 clear exactly when
+// hm > hT, and never borrows from the half above. A kept half has hm >= 1,
+// so its sign bit alone decides "negative". Non-finite kept halves are kept
+// but left out of the sum (as in the element-wise form, taken for them).
 template <bool TERNARY>
 __device__ __forceinline__ void keep8(const uint4 &v, uint32_t hT, int64_t k0, int64_t K,
                                       uint32_t &kb, uint32_t &sb, uint64_t &ks) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  kb = 0;
-  sb = 0;
-  double kd = 0.0;  // kept magnitudes: exact, as in sum_mag8
+  if (TERNARY) {
+    const uint32_t tc = (hT | 0x8000u) * 0x00010001u;
+    uint32_t kw[4], nw[4], kv[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t h = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
-    const uint32_t hm = h & 0x7FFFu;
-    uint32_t keep;
-    if (TERNARY) {
-      keep = hm > hT;
-      kd += keep && hm < 0x7C00u ? half_mag(hm) : 0.0;
-    } else {
-      keep = (k0 + i) < K;
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t hm2 = w[j] & MAG2;
+      kw[j] = ~(tc - hm2) & 0x80008000u;
+      nw[j] = w[j] & kw[j];
+      kv[j] = hm2 & ((kw[j] >> 15) * 0x7FFFu);
     }
-    const uint32_t neg = keep & (h >> 15) & (hm != 0u);
-    kb |= keep << i;
-    sb |= neg << i;
+    kb = gather_bit15(kw[0], kw[1], kw[2], kw[3]);
+    sb = gather_bit15(nw[0], nw[1], nw[2], nw[3]);
+    const double kd = f64_sum8(kv[0], kv[1], kv[2], kv[3]);
+    if (finite_f64(kd)) {
+      ks += units_of(kd);
+    } else {
+      bool unused = false;
+      ks += sum_mag8_nonfinite(make_uint4(kv[0], kv[1], kv[2], kv[3]), unused);
+    }
+  } else {
+    kb = 0;
+    sb = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t h = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+      const uint32_t keep = (k0 + i) < K;
+      kb |= keep << i;
+      sb |= (keep & (h >> 15) & ((h & 0x7FFFu) != 0u)) << i;
+    }
   }
-  if (TERNARY) ks += units_of(kd);
 }
 
 // E4M3 word k (k = 0..7) of a 32-element block in the tensor-core order: its
