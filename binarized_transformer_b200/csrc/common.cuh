@@ -22,17 +22,23 @@ constexpr uint64_t DRAIN_NS = 1000000000ull;
 #ifndef __CUDACC_RTC__
 // The >48 KB dynamic shared-memory opt-in of one kernel, made once per device
 // (the device current at the call). Only a success is remembered, so a call
-// that failed is retried on the next launch.
+// that failed is retried on the next launch. With max_carveout the kernel also
+// asks for the largest shared-memory carveout, so that an SM running one of
+// its CTAs keeps room for a CTA of the next kernel in the stream (left to
+// itself the driver may size the carveout for this kernel's CTA alone).
 class SmemOptIn {
  public:
   template <typename Kern>
-  cudaError_t operator()(Kern *kern, int bytes) {
+  cudaError_t operator()(Kern *kern, int bytes, bool max_carveout = false) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const bool cached = dev >= 0 && dev < kDevices;
     if (cached && set_[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && max_carveout)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess && cached) set_[dev].store(bytes, std::memory_order_release);
     return e;
   }

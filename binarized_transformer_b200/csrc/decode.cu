@@ -169,7 +169,8 @@ __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
 // compute threads then make the planes of every staged row: pass 1 sums the
 // magnitudes of all the round's rows (one partial per row and warp), pass 2
 // derives each row's threshold from them and writes the row's bits and kept
-// sums, and the row scales follow -- four barriers per round. Piece q (8
+// sums (and the popcount of each mask chunk), and the row scales follow --
+// three barriers per round. Piece q (8
 // halves) of a row belongs to thread q % 256; 16 consecutive threads cover
 // one 128-element chunk.
 template <bool FUSED>
@@ -265,6 +266,7 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
         uint4 *sA = reinterpret_cast<uint4 *>(smem + J.act_off);
         uint32_t *mrow = reinterpret_cast<uint32_t *>(sA + mm * nch);
         uint32_t *srow = reinterpret_cast<uint32_t *>(sA + J.M * nch + mm * nch);
+        int *prow = reinterpret_cast<int *>(sA + 2 * J.M * nch) + mm * nch;
         const uint4 *row = stage + off;
         uint64_t ks = 0, kn = 0;
         for (int st = 0; st < steps; ++st) {  // uniform trip count: store_chunk shuffles
@@ -275,7 +277,7 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
           if (p.ternary) keep8<true>(v, hT, k0, K, kb, sb, ks);
           else keep8<false>(v, hT, k0, K, kb, sb, ks);
           kn += __popc(kb);
-          store_chunk(kb, sb, mrow, srow, chunk, chunk < nch);
+          store_chunk(kb, sb, mrow, srow, chunk, chunk < nch, nullptr, prow);
         }
         ks = warp_sum_u64(ks);
         kn = warp_sum_u64(kn);
@@ -315,20 +317,13 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
       }
       ssc[mm] = row_scale(a, b);
     }
-    cbar();  // the staging area and the partial sums are free again
-  }
-  // popcounts of the mask chunks
-  for (int jj = 0; jj < p.njobs; ++jj) {
-    const DecodeJob &J = p.job[jj];
-    const uint4 *sA = reinterpret_cast<const uint4 *>(smem + J.act_off);
-    int *sP = reinterpret_cast<int *>(const_cast<uint4 *>(sA) + 2 * J.M * J.nchunks);
-    for (int idx = tid; idx < J.M * J.nchunks; idx += DC_CTHREADS) {
-      const uint4 v = sA[idx];
-      sP[idx] = __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
-    }
+    // The staging area and the partial sums are reused by the next round.
+    // After the last round no barrier is needed: the planes were complete at
+    // the barrier above, and the scales are read only by the fold warps,
+    // after the writer's warp has released its first fold table.
+    if (j < p.njobs) cbar();
   }
   if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
-  cbar();
 }
 
 // ------------------------------------------------------------------ kernel
@@ -337,12 +332,24 @@ __host__ __device__ __forceinline__ size_t dc_tab_d_bytes(int mr, int pitch) {
   return ((size_t)mr * DC_R * pitch * 2 + 15) / 16 * 16;
 }
 
+// Two CTAs per SM by registers: an SM running a CTA of this launch keeps room
+// for a CTA of the next kernel in the stream (416 threads x 80 registers, the
+// allocation of 74, would not fit twice in 64 K registers).
 template <int MR, bool FUSED>
-__global__ void __launch_bounds__(DC_THREADS, 1)
-k_decode(const __grid_constant__ DecodeBatch p, int32_t *d_status) {
+__global__ void __launch_bounds__(DC_THREADS, 2)
+k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
   extern __shared__ uint4 dc_smem4[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(dc_smem4);
   __shared__ DcBars bars;
+  // The launch parameters (1.4 KB) are copied to shared memory with one load
+  // per thread: read in place, the job lookups below would be chains of
+  // dependent constant-cache misses at the start of every launch.
+  __shared__ DecodeBatch p_s;
+  static_assert(sizeof(DecodeBatch) % 4 == 0, "copied as words");
+  for (int w = threadIdx.x; w < (int)(sizeof(DecodeBatch) / 4); w += DC_THREADS)
+    reinterpret_cast<uint32_t *>(&p_s)[w] = reinterpret_cast<const uint32_t *>(&pk)[w];
+  __syncthreads();
+  const DecodeBatch &p = p_s;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t stride = gridDim.x;
   uint8_t *ring = smem + p.ring_off;
@@ -551,7 +558,7 @@ static cudaError_t launch_decode_t(const DecodeBatch &p, size_t smem, int32_t *d
                                    cudaStream_t s) {
   auto kern = k_decode<MR, FUSED>;
   static SmemOptIn opt_in;
-  if (cudaError_t e = opt_in(kern, (int)smem)) return e;
+  if (cudaError_t e = opt_in(kern, (int)smem, true)) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -14,16 +14,16 @@
 // handed out round-robin; every ring below runs on across tile boundaries, so
 // the loads and MMAs of the next tile overlap the last groups and the stores
 // of the current one. Warp roles:
-//  * warp 12 (one thread) issues the TMA loads of each 128-column k-block:
+//  * warp 0 (one thread) issues the TMA loads of each 128-column k-block:
 //    128 tokens x 128 E4M3 bytes of activations (128-byte swizzle) and the
 //    weight rows' sign bits (16 bytes per row), into an 8-stage ring;
-//  * warps 0-3 expand the sign bits into E4M3 +-1 in TMEM (operand A, one TMEM
+//  * warps 2-5 expand the sign bits into E4M3 +-1 in TMEM (operand A, one TMEM
 //    lane per weight row, 4 buffers). Weight k + 8j of a 32-column block goes
 //    to byte j of word k, the order in which the activation packer writes its
 //    E4M3 bytes, so a word costs one shift and one LOP3;
-//  * warp 13 (one thread) issues 4 MMAs (M=128, N=128, K=32) per k-block into
+//  * warp 1 (one thread) issues 4 MMAs (M=128, N=128, K=32) per k-block into
 //    one of three fp32 accumulators in TMEM (one per weight group in flight);
-//  * warps 4-11 fold each finished group into running fp32 sums in registers
+//  * warps 6-13 fold each finished group into running fp32 sums in registers
 //    (two warps per TMEM lane quarter, 64 tokens each) and write Y at the end
 //    of a tile.
 // MMA issue blocks until the tensor pipe takes the instruction and the pipe
@@ -50,7 +50,14 @@ constexpr int TC_KB = 128;      // K elements per k-block = one 128-byte swizzle
 constexpr int TC_STAGES = 8;    // smem ring of (activations, weight bits) k-blocks
 constexpr int TC_ABUF = 4;      // expanded-weight buffers in TMEM
 constexpr int TC_DBUF = 3;      // fp32 accumulators in TMEM
-constexpr int TC_PRODUCER = 12, TC_ISSUER = 13;
+// Warps: 0 TMA, 1 MMA issue, 2-5 expand, 6-13 epilogue. A warp reaches the
+// TMEM lanes of quarter warp % 4 only, so the expand and epilogue warps cover
+// the four quarters by their index mod 4. The MMA issuer shares its SM
+// sub-partition with busy expand and epilogue warps; measured alone, its MMA
+// rate drops 3.6x when high-ILP warps compete for the same issue slots, so it
+// is the lowest-numbered warp there and the epilogue issues half as many FMA
+// instructions (two fp32 FMAs per instruction).
+constexpr int TC_PRODUCER = 0, TC_ISSUER = 1, TC_EXPAND0 = 2, TC_EPI0 = 6;
 constexpr int TC_THREADS = 14 * 32;
 constexpr int TC_X_BYTES = TC_BN * TC_KB;  // 16 KB of E4M3 activations per stage
 constexpr int TC_W_BYTES = TC_BM * 16;     // 2 KB of weight sign bits per stage
@@ -88,6 +95,17 @@ __device__ __forceinline__ bool tc_wait(TcBarriers *b, uint64_t *bar, uint32_t p
   if (mbar_wait(bar, parity, 2000000000ull)) return true;
   b->timeout = 1;
   return false;
+}
+
+// (y0, y1) = (fma(d0, a, y0), fma(d1, a, y1)) in one instruction: two IEEE
+// fp32 fused multiply-adds, the same results as two fmaf calls.
+__device__ __forceinline__ void fma2(float &y0, float &y1, float d0, float d1, float a) {
+  uint64_t yy, dd, aa, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(yy) : "f"(y0), "f"(y1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(dd) : "f"(d0), "f"(d1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(a));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(dd), "l"(aa), "l"(yy));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(r));
 }
 
 // Four E4M3 weights +-1 from the sign-bit word w: byte j is weight 8j + k
@@ -242,9 +260,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
       if (!mbar_wait(&bars->drain, 0, DRAIN_NS)) bars->undrained = 1;
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < TC_EPI0) {
     // ------------------------------------------------ weight bits -> E4M3 in TMEM
-    const int r = warp * 32 + lane;
+    const int qx = warp % 4, r = qx * 32 + lane;
     uint32_t g = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -273,7 +291,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
           v[8 * q + 6] = e4m3_pm1_tc<6>(wd[q]);
           v[8 * q + 7] = e4m3_pm1_tc<7>(wd[q]);
         }
-        tmem_st32(tmem_addr(tmem, warp * 32, TC_COL_A + b * 32), v);
+        tmem_st32(tmem_addr(tmem, qx * 32, TC_COL_A + b * 32), v);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -282,7 +300,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
     }
   } else {
     // ------------------------------------------------ epilogue: fold groups, write Y
-    const int h = (warp - 4) / 4, q = warp % 4, r = q * 32 + lane;
+    const int h = (warp - TC_EPI0) / 4, q = warp % 4, r = q * 32 + lane;
     uint32_t sg = 0, g0 = 0;  // groups and k-blocks of the tiles before this one
     bool ok = true;
     for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, g0 += KB) {
@@ -315,9 +333,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->d_empty[d]);
           }
+          if (seg == 0) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            y[c * 32 + i] = fmaf(__uint_as_float(dv[i]), alpha, seg > 0 ? y[c * 32 + i] : 0.0f);
+            for (int i = 0; i < 32; ++i) y[c * 32 + i] = 0.0f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            fma2(y[c * 32 + i], y[c * 32 + i + 1], __uint_as_float(dv[i]), __uint_as_float(dv[i + 1]), alpha);
           if (WANT_DOTS && seg == nseg - 1 && n < N) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {

@@ -166,7 +166,7 @@ __device__ __forceinline__ uint32_t e4m3_tc_word(uint32_t mw, uint32_t sw, int k
 // byte offset as its 8 elements).
 __device__ __forceinline__ void store_chunk(uint32_t kb, uint32_t sb, uint32_t *mrow,
                                             uint32_t *srow, int chunk, bool do_store,
-                                            uint8_t *e4m3_dst = nullptr) {
+                                            uint8_t *e4m3_dst = nullptr, int *popc_dst = nullptr) {
   const int l16 = threadIdx.x & 15;
   uint32_t mw = kb << (8 * (l16 & 3)), sw = sb << (8 * (l16 & 3));
   mw |= __shfl_xor_sync(FULL, mw, 1);
@@ -185,6 +185,7 @@ __device__ __forceinline__ void store_chunk(uint32_t kb, uint32_t sb, uint32_t *
   if (do_store && l16 == 0) {
     *reinterpret_cast<uint4 *>(mrow + 4 * chunk) = make_uint4(mw, m1, m2, m3);
     *reinterpret_cast<uint4 *>(srow + 4 * chunk) = make_uint4(sw, s1, s2, s3);
+    if (popc_dst) popc_dst[chunk] = __popc(mw) + __popc(m1) + __popc(m2) + __popc(m3);
   }
 }
 
