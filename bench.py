@@ -702,7 +702,7 @@ def decode_model_row(args, flush, hbm, emit, layers=32):
     graph = capture_graph(fused_step)
     t = _time_fn(graph.replay, max(3, args.steps), flush)
     emit("llama7b_decode_32_layers", t, nbytes=wbytes, tokens_per_s=round(1.0 / t, 1),
-         launches=layers * len(shapes), kernel="k_linear_decode (fused ternarize + GEMV)",
+         launches=layers * len(shapes), kernel="k_decode (fused ternarize + GEMV)",
          note="linear layers only")
 
 

@@ -257,11 +257,15 @@ cudaError_t launch_billm_pack(const float *W, int64_t ldW, int split, const bill
 // add per weight and row of X, plus a few multiply-adds for the ~10% of
 // columns that are sparse or salient. Partial sums are per 128-column block
 // (fp32 error ~128 * 2^-24 of the block's magnitude), folded into y per block.
-constexpr int BR_THREADS = 256, BR_SPLIT = 4, BR_ROWS = BR_THREADS / BR_SPLIT;
+constexpr int BR_SPLIT = 4;  // threads per weight row
+// 256 threads (64 rows) per CTA for MP <= 4; 512 (128 rows) for larger MP,
+// whose inner loop is latency-bound at 8 warps per SM.
+template <int MP>
+constexpr int br_threads() { return MP <= 4 ? 256 : 512; }
 constexpr size_t BR_SMEM_BUDGET = 160 * 1024;
 constexpr int BR_MAX_NB = 40960 / 128;
 
-template <int MP>
+template <int MP, int BR_THREADS = br_threads<MP>(), int BR_ROWS = BR_THREADS / BR_SPLIT>
 __global__ void __launch_bounds__(BR_THREADS)
 k_billm_rows(const uint16_t *__restrict__ X, int64_t M, int64_t ldX, const uint32_t *__restrict__ sign,
              const uint32_t *__restrict__ gmap, const uint8_t *__restrict__ res,
@@ -442,6 +446,7 @@ template <int MP>
 static cudaError_t launch_br_t(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,
                                float *Y, int64_t ldY, int32_t *d_status, cudaStream_t s) {
   auto kern = k_billm_rows<MP>;
+  constexpr int BR_THREADS = br_threads<MP>(), BR_ROWS = BR_THREADS / BR_SPLIT;
   const int slice = br_slice(MP, W->K);
   const size_t smem = (size_t)(slice / 128) * (128 * MP + 4 + MP) * 4 +
                       (size_t)(W->K / 128) * W->n_sal;
@@ -463,10 +468,11 @@ static cudaError_t launch_br_t(const uint16_t *X, int64_t M, int64_t ldX, const 
 cudaError_t launch_billm_gemm(const uint16_t *X, int64_t M, int64_t ldX, const billm_weights *W,
                               float *Y, int64_t ldY, int32_t *d_status, cudaStream_t s) {
   if (M == 0 || W->N == 0) return cudaSuccess;
-  // M <= 4 on CUDA cores (the weight rebuild of the tensor-core kernel costs
-  // as much at M = 2 as at M = 512); larger M on tensor cores, when X
+  // M <= 8 on CUDA cores (the weight rebuild of the tensor-core kernel costs
+  // as much at M = 2 as at M = 512: measured 648 us at M = 2..16 against 155,
+  // 355 and 425 us here for M = 2, 4, 8); larger M on tensor cores, when X
   // satisfies the TMA alignment rules.
-  if (M > 4) {
+  if (M > 8) {
     const cudaError_t e = launch_billm_gemm_tc(X, M, ldX, W, Y, ldY, d_status, s);
     if (e != cudaErrorNotSupported) return e;
   }

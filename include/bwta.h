@@ -327,11 +327,11 @@ int billm_pack_weights(const float *W, int64_t ldW, int split, const billm_weigh
  * residual plane, non-salient weights in two groups with their own scales):
  * Y[m][n] = sum_k x[m][k] * what[n][k], the same real value as the per-block form
  *   alpha_c*sum_C b x + alpha_sp*sum_S b x + alpha1*sum_sal b1 x + alpha2*sum_sal b2 x.
- *  M <= 4: CUDA cores, one 128-column block at a time (fp32 sums per block,
- *  folded into Y per block). M > 4 with X 16-byte aligned and ldX % 8 == 0:
+ *  M <= 8: CUDA cores, one 128-column block at a time (fp32 sums per block,
+ *  folded into Y per block). M > 8 with X 16-byte aligned and ldX % 8 == 0:
  *  tensor cores; each weight is rebuilt as what * 2^E (E per weight row)
  *  split into fp16 hi + lo, and X*hi + X*lo accumulates in fp32 over all of
- *  K. Other M > 4: CUDA cores as for M <= 4.
+ *  K. Other M > 8: CUDA cores as for M <= 8.
  *  Accuracy: fp32 sums, so the error is not bounded by a fixed fraction of
  *  sum_k |x_k what_k| in the worst case (about K * 2^-24 of it for the
  *  tensor-core path, 128 * 2^-24 per block for the CUDA-core paths); measured

@@ -402,11 +402,12 @@ def test_billm_searched_split_full_config_rows():
     assert_close_rel(Y[:, rows], yref, mag, what="billm searched split")
 
 
-@pytest.mark.parametrize("N,K,M", [(200, 384, 300), (129, 128, 70), (64, 1024, 5), (300, 256, 257),
-                                   (64, 1024, 2), (130, 384, 3), (33, 256, 4)])
+@pytest.mark.parametrize("N,K,M", [(200, 384, 300), (129, 128, 70), (64, 1024, 9), (300, 256, 257),
+                                   (64, 1024, 2), (130, 384, 3), (33, 256, 4), (200, 384, 7), (65, 512, 8)])
 def test_billm_tc_shapes(N, K, M):
-    """Tensor-core BiLLM path (M > 4): ragged token tiles (64 and 256), ragged
-    weight-row tiles, odd block counts; M = 2..4 take the CUDA-core kernel."""
+    """Tensor-core BiLLM path (M > 8): ragged token tiles (64 and 256), ragged
+    weight-row tiles, odd block counts; M = 2..8 take the CUDA-core kernel
+    (512 threads for M > 4)."""
     W = workloads.latent_laplace((N, K), 0.01, 11, N, K)
     X = workloads.edge_acts(M, K, "student", tag=N + K)
     Wq = bt.billm_pack_weights(dev(W), n_sal=8, split=True)
