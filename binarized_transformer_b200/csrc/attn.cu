@@ -266,7 +266,8 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
     }
     // scores times the softmax factor, and the row max
     float mx = -INFINITY;
-    for (int64_t j = l; j < Lk; j += 32) {
+    const int lk = (int)Lk;
+    for (int j = l; j < lk; j += 32) {
       int d = 0;
       if (NW != 4) {
         d = tern_dot<NW>(qa[0], qb[0], sKm[j], sKs[j]);
@@ -282,7 +283,7 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
     double z = 0.0;
-    for (int64_t j = l; j < Lk; j += 32) {
+    for (int j = l; j < lk; j += 32) {
       const float e = expf(xw[j] - mx);
       xw[j] = e;
       z += (double)e;
@@ -290,28 +291,32 @@ k_attn_softmax_pack(const uint32_t *__restrict__ qm, const uint32_t *__restrict_
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
     const double cut = z * thr;
+    // For an fp32 value e, e > cut exactly when e > cut rounded down to fp32
+    // (the largest fp32 not above cut): the keep test runs in fp32.
+    const float cut32 = __double2float_rd(cut);
     // keep bits: key j = 32t + l is bit l of mask word t
     double ksum = 0.0;
     int kn = 0;
     uint32_t *mrow = pm + (bh * Lq + i) * ldp, *srow = ps + (bh * Lq + i) * ldp;
     uint32_t myword = 0;  // lane l keeps mask word l (of each group of 32 words)
-    for (int64_t t = 0; t * 32 < Lk; ++t) {
-      const int64_t j = t * 32 + l;
-      const double e = j < Lk ? (double)xw[j] : 0.0;
-      const bool keep = e > cut;
+    const int nt = (lk + 31) / 32;
+    for (int t = 0; t < nt; ++t) {
+      const int j = t * 32 + l;
+      const float e = j < lk ? xw[j] : 0.0f;
+      const bool keep = e > cut32;
       const uint32_t word = __ballot_sync(FULL, keep);
-      if (keep) ksum += e;
+      if (keep) ksum += (double)e;
       kn += keep;
       if (l == (t & 31)) myword = word;
-      if ((t & 31) == 31 || (t + 1) * 32 >= Lk) {  // one coalesced store per 32 words
-        const int64_t t0 = t & ~(int64_t)31;
+      if ((t & 31) == 31 || t + 1 == nt) {  // one coalesced store per 32 words
+        const int t0 = t & ~31;
         if (t0 + l <= t) {
           mrow[t0 + l] = myword;
           srow[t0 + l] = 0u;
         }
       }
     }
-    for (int t = (int)((Lk + 31) / 32) + l; t < ldp; t += 32) {  // padding words
+    for (int t = nt + l; t < ldp; t += 32) {  // padding words
       mrow[t] = 0u;
       srow[t] = 0u;
     }
