@@ -60,7 +60,7 @@ constexpr int DC_MAX_CHUNKS = 128;               // K <= 16384
 constexpr size_t DC_MAX_ACT_SMEM = 48 * 1024;
 constexpr size_t DC_RING_BUDGET = 56 * 1024;     // bytes of weight tiles in flight per CTA
 constexpr size_t DC_TAB_BUDGET = 48 * 1024;      // fold tables (at least two)
-constexpr int DC_STAGE_ROWS_BYTES = 24 * 1024;   // fused: fp16 rows staged per round
+constexpr int DC_STAGE_ROWS_BYTES = 48 * 1024;   // fused: fp16 rows staged per round
 constexpr int DC_ROUND_ROWS = 32;                // fused: at most this many rows per round
 static_assert(DC_R == 16 && DC_RPW * DC_WARPS == DC_R, "fold lanes 0..15, two rows per warp");
 
