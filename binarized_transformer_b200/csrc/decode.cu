@@ -126,12 +126,22 @@ __device__ __forceinline__ int dc_job_of(const DecodeBatch &p, int64_t tile) {
 // The dot warps' barrier (the fold and copy warps never take part).
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, %0;" ::"n"(DC_CTHREADS) : "memory"); }
 
-// Bulk copy global -> this CTA's shared memory (no multicast), completing on `bar`.
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+// L2 policy for data read once: evict it first, so the weight stream does not
+// push the activations and outputs of neighbouring launches out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// Bulk copy global -> this CTA's shared memory (no multicast), completing on
+// `bar`, under the L2 policy `pol`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                          uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, "
+      "[%3], %4;" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
       : "memory");
 }
 
@@ -373,6 +383,7 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
     // ------------------------------------------------ copy warp
     if (lane == 0) {
       if (!p.ready) pdl_wait();  // weights may still be written by the previous kernel
+      const uint64_t pol = l2_evict_first();  // every weight byte is read once per launch
       int i = 0;
       for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += stride, ++i) {
         const int s = i % p.stages;
@@ -387,8 +398,8 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
         float *sdst = reinterpret_cast<float *>(st + p.stage_bits);
         for (uint32_t q = s16 / 4; q < sbytes / 4; ++q) sdst[q] = __ldg(J.ws + n0 * J.G + q);
         mbar_arrive_expect_tx(&bars.full[s], bbytes + s16);
-        bulk_load(st, J.wb + n0 * J.ldw, bbytes, &bars.full[s]);
-        if (s16) bulk_load(sdst, J.ws + n0 * J.G, s16, &bars.full[s]);
+        bulk_load(st, J.wb + n0 * J.ldw, bbytes, &bars.full[s], pol);
+        if (s16) bulk_load(sdst, J.ws + n0 * J.G, s16, &bars.full[s], pol);
       }
       // Copies still in flight (after a timeout) land before the CTA exits; a
       // stage is refilled only after its previous copy was consumed, so only
