@@ -117,12 +117,6 @@ __device__ __forceinline__ JobActs job_acts(uint8_t *smem, const DecodeJob &J) {
   return {a, s, p, reinterpret_cast<float *>(p + J.M * J.nchunks)};
 }
 
-__device__ __forceinline__ int dc_job_of(const DecodeBatch &p, int64_t tile) {
-  int j = 0;
-  while (j + 1 < p.njobs && tile >= p.job[j + 1].tile0) ++j;
-  return j;
-}
-
 // The dot warps' barrier (the fold and copy warps never take part).
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, %0;" ::"n"(DC_CTHREADS) : "memory"); }
 
@@ -384,22 +378,37 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
     if (lane == 0) {
       if (!p.ready) pdl_wait();  // weights may still be written by the previous kernel
       const uint64_t pol = l2_evict_first();  // every weight byte is read once per launch
-      int i = 0;
+      // This single thread is the CTA's only source of copies: its loop keeps
+      // the stage index and round in counters and the current job's fields
+      // in registers (a CTA meets each job's tiles in one run).
+      int i = 0, s = 0, j = -1;
+      uint32_t round = 0;
+      int64_t tend = 0, jt0 = 0, jN = 0, jldw = 0, jG = 0;
+      const uint32_t *jwb = nullptr;
+      const float *jws = nullptr;
+      bool jY = false;
       for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += stride, ++i) {
-        const int s = i % p.stages;
-        if (i >= p.stages && !dc_wait(bars, &bars.empty[s], ((i / p.stages) - 1) & 1)) break;
-        const DecodeJob &J = p.job[dc_job_of(p, tile)];
-        const int64_t n0 = (tile - J.tile0) * DC_R;
-        const int64_t rows = J.N - n0 < DC_R ? J.N - n0 : DC_R;
+        if (i >= p.stages && !dc_wait(bars, &bars.empty[s], (round & 1) ^ 1)) break;
+        while (tile >= tend) {
+          const DecodeJob &J = p.job[++j];
+          jt0 = J.tile0, jN = J.N, jldw = J.ldw, jG = J.G, jwb = J.wb, jws = J.ws, jY = J.Y != nullptr;
+          tend = j + 1 < p.njobs ? p.job[j + 1].tile0 : p.ntiles;
+        }
+        const int64_t n0 = (tile - jt0) * DC_R;
+        const int64_t rows = jN - n0 < DC_R ? jN - n0 : DC_R;
         uint8_t *st = ring + (size_t)s * p.stage_bytes;
-        const uint32_t bbytes = (uint32_t)(rows * J.ldw * 4);
-        const uint32_t sbytes = J.Y ? (uint32_t)(rows * J.G * 4) : 0u, s16 = sbytes & ~15u;
+        const uint32_t bbytes = (uint32_t)(rows * jldw * 4);
+        const uint32_t sbytes = jY ? (uint32_t)(rows * jG * 4) : 0u, s16 = sbytes & ~15u;
         // a scale tail that is not a whole 16 bytes: plain loads (published by the arrive)
         float *sdst = reinterpret_cast<float *>(st + p.stage_bits);
-        for (uint32_t q = s16 / 4; q < sbytes / 4; ++q) sdst[q] = __ldg(J.ws + n0 * J.G + q);
+        for (uint32_t q = s16 / 4; q < sbytes / 4; ++q) sdst[q] = __ldg(jws + n0 * jG + q);
         mbar_arrive_expect_tx(&bars.full[s], bbytes + s16);
-        bulk_load(st, J.wb + n0 * J.ldw, bbytes, &bars.full[s], pol);
-        if (s16) bulk_load(sdst, J.ws + n0 * J.G, s16, &bars.full[s], pol);
+        bulk_load(st, jwb + n0 * jldw, bbytes, &bars.full[s], pol);
+        if (s16) bulk_load(sdst, jws + n0 * jG, s16, &bars.full[s], pol);
+        if (++s == p.stages) {
+          s = 0;
+          ++round;
+        }
       }
       // Copies still in flight (after a timeout) land before the CTA exits; a
       // stage is refilled only after its previous copy was consumed, so only
@@ -420,12 +429,17 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
     // each table's barriers are waited on in order by one warp (a parity
     // wait never sees a phase two ahead).
     const int f = warp - DC_WARPS;
-    int i = f;
+    int b = f, j = -1;
+    uint32_t round = 0;
+    int64_t tend = 0;
     for (int64_t tile = blockIdx.x + (int64_t)f * stride; f < p.nfold && tile < p.ntiles;
-         tile += (int64_t)p.nfold * stride, i += p.nfold) {
-      const int b = i % p.ntabs;
-      if (!__all_sync(FULL, dc_wait(bars, &bars.tfull[b], (i / p.ntabs) & 1))) break;
-      const DecodeJob &J = p.job[dc_job_of(p, tile)];
+         tile += (int64_t)p.nfold * stride) {
+      if (!__all_sync(FULL, dc_wait(bars, &bars.tfull[b], round & 1))) break;
+      while (tile >= tend) {
+        ++j;
+        tend = j + 1 < p.njobs ? p.job[j + 1].tile0 : p.ntiles;
+      }
+      const DecodeJob &J = p.job[j];
       const JobActs acts = job_acts(smem, J);
       const uint8_t *tab = smem + p.tab_off + (size_t)b * p.tab_bytes;
       const int nch = J.nchunks, gc = J.gchunks;
@@ -500,6 +514,11 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.tempty[b]);
+      b += p.nfold;  // tables f, f + nfold, ... (ntabs is a multiple of nfold)
+      if (b >= p.ntabs) {
+        b -= p.ntabs;
+        ++round;
+      }
     }
     return;
   }
@@ -508,32 +527,41 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
   pdl_wait();  // activations follow the previous kernel in the stream
   dc_setup_acts<FUSED>(p, smem, d_status);
 
-  int i = 0;
+  // stage and table indices and their rounds in counters; the current job's
+  // fields in registers, reloaded when the tiles move into the next job
+  int i = 0, s = 0, b = 0, j = -1;
+  uint32_t sround = 0, bround = 0;
+  int64_t tend = 0, jldw = 0, jG = 0;
+  int nch = 0, gc = 1, jM = 0;
+  bool jY = false;
+  JobActs acts = {};
   for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += stride, ++i) {
-    const int s = i % p.stages, b = i % p.ntabs;
-    const DecodeJob &J = p.job[dc_job_of(p, tile)];
-    bool ok = dc_wait(bars, &bars.full[s], (i / p.stages) & 1);
-    if (ok && i >= p.ntabs) ok = dc_wait(bars, &bars.tempty[b], ((i / p.ntabs) - 1) & 1);
+    while (tile >= tend) {
+      const DecodeJob &J = p.job[++j];
+      jldw = J.ldw, jG = J.G, nch = J.nchunks, gc = J.gchunks, jM = J.M, jY = J.Y != nullptr;
+      acts = job_acts(smem, J);
+      tend = j + 1 < p.njobs ? p.job[j + 1].tile0 : p.ntiles;
+    }
+    bool ok = dc_wait(bars, &bars.full[s], sround & 1);
+    if (ok && i >= p.ntabs) ok = dc_wait(bars, &bars.tempty[b], (bround & 1) ^ 1);
     if (!__all_sync(FULL, ok)) break;  // warp-uniform: the loop below synchronizes the warp
-    const JobActs acts = job_acts(smem, J);
     const uint8_t *st = ring + (size_t)s * p.stage_bytes;
     uint8_t *tab = smem + p.tab_off + (size_t)b * p.tab_bytes;
     int16_t *td = reinterpret_cast<int16_t *>(tab);
     float *ta = reinterpret_cast<float *>(tab + dc_tab_d_bytes(MR, p.pitch));
-    const int nch = J.nchunks, gc = J.gchunks;
     // integer dots of this warp's rows with every activation row
 #pragma unroll
     for (int rr = 0; rr < DC_RPW; ++rr) {
       const int r = warp * DC_RPW + rr;
-      const uint4 *bits = reinterpret_cast<const uint4 *>(st + (size_t)r * J.ldw * 4);
-      const float *sc = reinterpret_cast<const float *>(st + p.stage_bits) + r * J.G;
+      const uint4 *bits = reinterpret_cast<const uint4 *>(st + (size_t)r * jldw * 4);
+      const float *sc = reinterpret_cast<const float *>(st + p.stage_bits) + r * jG;
       for (int c = lane; c < nch; c += 32) {
         const uint4 w = bits[c];
-        ta[r * p.pitch + c] = J.Y ? sc[gc == 1 ? c : c / gc] : 0.0f;
+        ta[r * p.pitch + c] = jY ? sc[gc == 1 ? c : c / gc] : 0.0f;
 #pragma unroll
         for (int m = 0; m < MR; ++m) {
           int d = 0;
-          if (m < J.M) {
+          if (m < jM) {
             const uint4 A = acts.sA[m * nch + c], S = acts.sS[m * nch + c];
             d = acts.sP[m * nch + c] -
                 2 * popc4_csa(lop3_and_xor(A.x, S.x, w.x), lop3_and_xor(A.y, S.y, w.y),
@@ -547,6 +575,14 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
     if (lane == 0) {
       mbar_arrive(&bars.empty[s]);
       mbar_arrive(&bars.tfull[b]);
+    }
+    if (++s == p.stages) {
+      s = 0;
+      ++sround;
+    }
+    if (++b == p.ntabs) {
+      b = 0;
+      ++bround;
     }
   }
   if (lane == 0 && warp == 0 && *(volatile int32_t *)&bars.timeout)
