@@ -59,6 +59,9 @@ constexpr int DC_MAX_JOBS = 8;
 constexpr int DC_MAX_CHUNKS = 128;               // K <= 16384
 constexpr size_t DC_MAX_ACT_SMEM = 48 * 1024;
 constexpr size_t DC_RING_BUDGET = 56 * 1024;     // bytes of weight tiles in flight per CTA
+#ifndef DC_PF_BYTES
+#define DC_PF_BYTES (128 * 1024)                  // bytes of weight tiles prefetched into L2 per CTA
+#endif
 constexpr size_t DC_TAB_BUDGET = 48 * 1024;      // fold tables (at least two)
 constexpr int DC_STAGE_ROWS_BYTES = 48 * 1024;   // fused: fp16 rows staged per round
 constexpr int DC_ROUND_ROWS = 32;                // fused: at most this many rows per round
@@ -88,6 +91,7 @@ struct DecodeBatch {
   int64_t ntiles;
   int njobs, ternary, ready;
   int stages, stage_bits, stage_bytes;  // copy ring: depth, bytes of sign words / of a stage
+  int pf_ahead;                         // tiles prefetched into L2 ahead of the ring
   int ring_off;
   int ntabs, nfold;                     // fold tables (a multiple of nfold), active fold warps
   int tab_off, tab_bytes, pitch;        // fold tables (pitch odd, in elements)
@@ -127,6 +131,33 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
+
+// Bulk prefetch of global memory into L2 under the policy `pol` (no
+// completion to track: a later copy of the same bytes finds them in L2).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes, uint64_t pol) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(src), "r"(bytes),
+               "l"(pol)
+               : "memory");
+}
+
+// The job a tile belongs to, with the fields the copy thread needs, kept in
+// registers while tiles advance through the jobs in order.
+struct DcCursor {
+  int j = -1;
+  int64_t tend = 0, t0 = 0, N = 0, ldw = 0, G = 0;
+  const uint32_t *wb = nullptr;
+  const float *ws = nullptr;
+  bool Y = false;
+  __device__ __forceinline__ void seek(const DecodeBatch &p, int64_t tile) {
+    while (tile >= tend) {
+      const DecodeJob &J = p.job[++j];
+      t0 = J.tile0, N = J.N, ldw = J.ldw, G = J.G, wb = J.wb, ws = J.ws, Y = J.Y != nullptr;
+      tend = j + 1 < p.njobs ? p.job[j + 1].tile0 : p.ntiles;
+    }
+  }
+  // rows of the tile that starts at row n0 (the job's last tile may be short)
+  __device__ __forceinline__ int64_t rows(int64_t n0) const { return N - n0 < DC_R ? N - n0 : DC_R; }
+};
 
 // Bulk copy global -> this CTA's shared memory (no multicast), completing on
 // `bar`, under the L2 policy `pol`.
@@ -380,34 +411,41 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
       const uint64_t pol = l2_evict_first();  // every weight byte is read once per launch
       // This single thread is the CTA's only source of copies: its loop keeps
       // the stage index and round in counters and the current job's fields
-      // in registers (a CTA meets each job's tiles in one run).
-      int i = 0, s = 0, j = -1;
+      // in registers (a CTA meets each job's tiles in one run). The ring holds
+      // `stages` tiles; a second cursor keeps the next `pf_ahead` tiles on
+      // their way into L2 (bulk prefetches, no shared memory), so that more
+      // bytes per SM are in flight than the ring can hold and a refilled
+      // stage finds its bytes in L2.
+      int i = 0, s = 0;
       uint32_t round = 0;
-      int64_t tend = 0, jt0 = 0, jN = 0, jldw = 0, jG = 0;
-      const uint32_t *jwb = nullptr;
-      const float *jws = nullptr;
-      bool jY = false;
+      DcCursor c, pc;
+      int64_t ptile = blockIdx.x + (int64_t)p.stages * stride;
+      int pi = p.stages;
       for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += stride, ++i) {
         if (i >= p.stages && !dc_wait(bars, &bars.empty[s], (round & 1) ^ 1)) break;
-        while (tile >= tend) {
-          const DecodeJob &J = p.job[++j];
-          jt0 = J.tile0, jN = J.N, jldw = J.ldw, jG = J.G, jwb = J.wb, jws = J.ws, jY = J.Y != nullptr;
-          tend = j + 1 < p.njobs ? p.job[j + 1].tile0 : p.ntiles;
-        }
-        const int64_t n0 = (tile - jt0) * DC_R;
-        const int64_t rows = jN - n0 < DC_R ? jN - n0 : DC_R;
+        c.seek(p, tile);
+        const int64_t n0 = (tile - c.t0) * DC_R;
+        const int64_t rows = c.rows(n0);
         uint8_t *st = ring + (size_t)s * p.stage_bytes;
-        const uint32_t bbytes = (uint32_t)(rows * jldw * 4);
-        const uint32_t sbytes = jY ? (uint32_t)(rows * jG * 4) : 0u, s16 = sbytes & ~15u;
+        const uint32_t bbytes = (uint32_t)(rows * c.ldw * 4);
+        const uint32_t sbytes = c.Y ? (uint32_t)(rows * c.G * 4) : 0u, s16 = sbytes & ~15u;
         // a scale tail that is not a whole 16 bytes: plain loads (published by the arrive)
         float *sdst = reinterpret_cast<float *>(st + p.stage_bits);
-        for (uint32_t q = s16 / 4; q < sbytes / 4; ++q) sdst[q] = __ldg(jws + n0 * jG + q);
+        for (uint32_t q = s16 / 4; q < sbytes / 4; ++q) sdst[q] = __ldg(c.ws + n0 * c.G + q);
         mbar_arrive_expect_tx(&bars.full[s], bbytes + s16);
-        bulk_load(st, jwb + n0 * jldw, bbytes, &bars.full[s], pol);
-        if (s16) bulk_load(sdst, jws + n0 * jG, s16, &bars.full[s], pol);
+        bulk_load(st, c.wb + n0 * c.ldw, bbytes, &bars.full[s], pol);
+        if (s16) bulk_load(sdst, c.ws + n0 * c.G, s16, &bars.full[s], pol);
         if (++s == p.stages) {
           s = 0;
           ++round;
+        }
+        // once the ring's first fill is out, keep tiles i+1 .. i+pf_ahead prefetched
+        for (; i + 1 >= p.stages && pi <= i + p.pf_ahead && ptile < p.ntiles; ptile += stride, ++pi) {
+          pc.seek(p, ptile);
+          const int64_t m0 = (ptile - pc.t0) * DC_R, prow = pc.rows(m0);
+          bulk_prefetch_l2(pc.wb + m0 * pc.ldw, (uint32_t)(prow * pc.ldw * 4), pol);
+          const uint32_t ps16 = pc.Y ? (uint32_t)(prow * pc.G * 4) & ~15u : 0u;
+          if (ps16) bulk_prefetch_l2(pc.ws + m0 * pc.G, ps16, pol);
         }
       }
       // Copies still in flight (after a timeout) land before the CTA exits; a
@@ -549,26 +587,39 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
     uint8_t *tab = smem + p.tab_off + (size_t)b * p.tab_bytes;
     int16_t *td = reinterpret_cast<int16_t *>(tab);
     float *ta = reinterpret_cast<float *>(tab + dc_tab_d_bytes(MR, p.pitch));
-    // integer dots of this warp's rows with every activation row
+    // integer dots of this warp's two rows with every activation row. The
+    // rows share each activation chunk's loads, and all of a chunk's loads are
+    // issued before its stores (a store to the table may alias a later load,
+    // so the compiler keeps them in program order).
+    static_assert(DC_RPW == 2, "two rows per dot warp");
+    const int r0 = warp * DC_RPW;
+    const uint4 *bits0 = reinterpret_cast<const uint4 *>(st + (size_t)r0 * jldw * 4);
+    const uint4 *bits1 = reinterpret_cast<const uint4 *>(st + (size_t)(r0 + 1) * jldw * 4);
+    const float *sc0 = reinterpret_cast<const float *>(st + p.stage_bits) + r0 * jG;
+    const float *sc1 = sc0 + jG;
+    for (int c = lane; c < nch; c += 32) {
+      const uint4 w0 = bits0[c], w1 = bits1[c];
+      const int g = gc == 1 ? c : c / gc;
+      const float a0 = jY ? sc0[g] : 0.0f, a1 = jY ? sc1[g] : 0.0f;
+      int d0[MR], d1[MR];
 #pragma unroll
-    for (int rr = 0; rr < DC_RPW; ++rr) {
-      const int r = warp * DC_RPW + rr;
-      const uint4 *bits = reinterpret_cast<const uint4 *>(st + (size_t)r * jldw * 4);
-      const float *sc = reinterpret_cast<const float *>(st + p.stage_bits) + r * jG;
-      for (int c = lane; c < nch; c += 32) {
-        const uint4 w = bits[c];
-        ta[r * p.pitch + c] = jY ? sc[gc == 1 ? c : c / gc] : 0.0f;
-#pragma unroll
-        for (int m = 0; m < MR; ++m) {
-          int d = 0;
-          if (m < jM) {
-            const uint4 A = acts.sA[m * nch + c], S = acts.sS[m * nch + c];
-            d = acts.sP[m * nch + c] -
-                2 * popc4_csa(lop3_and_xor(A.x, S.x, w.x), lop3_and_xor(A.y, S.y, w.y),
-                              lop3_and_xor(A.z, S.z, w.z), lop3_and_xor(A.w, S.w, w.w));
-          }
-          td[(m * DC_R + r) * p.pitch + c] = (int16_t)d;
+      for (int m = 0; m < MR; ++m) {
+        d0[m] = d1[m] = 0;
+        if (m < jM) {
+          const uint4 A = acts.sA[m * nch + c], S = acts.sS[m * nch + c];
+          const int P = acts.sP[m * nch + c];
+          d0[m] = P - 2 * popc4_csa(lop3_and_xor(A.x, S.x, w0.x), lop3_and_xor(A.y, S.y, w0.y),
+                                    lop3_and_xor(A.z, S.z, w0.z), lop3_and_xor(A.w, S.w, w0.w));
+          d1[m] = P - 2 * popc4_csa(lop3_and_xor(A.x, S.x, w1.x), lop3_and_xor(A.y, S.y, w1.y),
+                                    lop3_and_xor(A.z, S.z, w1.z), lop3_and_xor(A.w, S.w, w1.w));
         }
+      }
+      ta[r0 * p.pitch + c] = a0;
+      ta[(r0 + 1) * p.pitch + c] = a1;
+#pragma unroll
+      for (int m = 0; m < MR; ++m) {
+        td[(m * DC_R + r0) * p.pitch + c] = (int16_t)d0[m];
+        td[(m * DC_R + r0 + 1) * p.pitch + c] = (int16_t)d1[m];
       }
     }
     __syncwarp();
@@ -668,6 +719,8 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
   p.stage_bytes = (int)((p.stage_bits + DC_R * G_max * 4 + 15) / 16 * 16);
   p.stages = (int)std::min<size_t>(DC_MAX_STAGES,
                                    std::max<size_t>(2, DC_RING_BUDGET / (size_t)p.stage_bytes));
+  // L2 prefetch window: about DC_PF_BYTES of tiles per CTA beyond the ring
+  p.pf_ahead = (int)(DC_PF_BYTES / (size_t)p.stage_bytes);
   p.ring_off = (int)act;
   const size_t ring = (size_t)p.stages * p.stage_bytes;
   // fold tables, then (fused) the staging area and partial sums over them
