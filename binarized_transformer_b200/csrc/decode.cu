@@ -96,7 +96,7 @@ struct DecodeBatch {
   int ntabs, nfold;                     // fold tables (a multiple of nfold), active fold warps
   int tab_off, tab_bytes, pitch;        // fold tables (pitch odd, in elements)
   int stage_off, stage_pieces;          // fused: fp16 staging area (over the fold tables)
-  int red_off;                          // fused: per-row partial sums (over the fold tables)
+  int red_off;                          // fused: per-row partial sums (after tables and staging)
 };
 
 struct DcBars {
@@ -189,11 +189,16 @@ __device__ __forceinline__ bool dc_wait(DcBars &b, uint64_t *bar, uint32_t parit
 }
 
 // ------------------------------------------------------------- activations
-// Warp sum of a uint64 (every lane gets the total).
+// Warp sum of a uint64, modulo 2^64 like a plain sum (every lane gets the
+// total): three 22-bit limbs summed by independent redux.sync instructions
+// (32 limbs of 22 bits cannot overflow 32), in place of a chain of ten
+// dependent 32-bit shuffles.
 __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-  return v;
+  constexpr uint64_t L22 = (1u << 22) - 1;
+  const uint64_t lo = __reduce_add_sync(FULL, (uint32_t)(v & L22));
+  const uint64_t mid = __reduce_add_sync(FULL, (uint32_t)((v >> 22) & L22));
+  const uint64_t hi = __reduce_add_sync(FULL, (uint32_t)(v >> 44));
+  return lo + (mid << 22) + (hi << 44);
 }
 
 // Planes of every job into shared memory: copied (bit-plane input) or made
@@ -265,8 +270,10 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
         ++j;
       }
     }
+    // Each thread reads back only the pieces it staged itself (piece q of
+    // every row is staged and read by thread q % 256), so its own wait is
+    // the only ordering pass 1 needs.
     cp_async_wait_all();
-    cbar();
     // pass 1: magnitude sums of every staged row
     {
       int off = 0;
@@ -315,7 +322,7 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
           store_chunk(kb, sb, mrow, srow, chunk, chunk < nch, nullptr, prow);
         }
         ks = warp_sum_u64(ks);
-        kn = warp_sum_u64(kn);
+        kn = __reduce_add_sync(FULL, (uint32_t)kn);  // at most K kept elements
         if (lane == 0) {
           red_k[r * DC_WARPS + wid] = ks;
           red_n[r * DC_WARPS + wid] = kn;
@@ -723,11 +730,13 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
   p.pf_ahead = (int)(DC_PF_BYTES / (size_t)p.stage_bytes);
   p.ring_off = (int)act;
   const size_t ring = (size_t)p.stages * p.stage_bytes;
-  // fold tables, then (fused) the staging area and partial sums over them
+  // fold tables; fused: the staging area over them, then the partial sums
+  // after both (read by the scale threads after the last barrier of the
+  // setup, while other warps may already be writing fold tables)
   p.pitch = nch_max | 1;
   p.tab_bytes = (int)((dc_tab_d_bytes(mr, p.pitch) + (size_t)DC_R * p.pitch * 4 + 15) / 16 * 16);
   p.tab_off = (int)(act + ring);
-  size_t over = 0;
+  size_t stage = 0, red = 0;
   if (fused) {  // every staged row fits; as many rows per round as the staging area holds
     size_t rows_bytes = 0, row_max = 0;
     for (int i = 0; i < nj; ++i) {
@@ -735,18 +744,19 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
       rows_bytes += rb * p.job[i].M;
       row_max = std::max(row_max, rb);
     }
-    const size_t stage = std::max(row_max, std::min(rows_bytes, (size_t)DC_STAGE_ROWS_BYTES));
+    stage = std::max(row_max, std::min(rows_bytes, (size_t)DC_STAGE_ROWS_BYTES));
     p.stage_off = p.tab_off;
     p.stage_pieces = (int)(stage / 16);
-    p.red_off = (int)(p.tab_off + stage);
-    over = stage + (size_t)3 * DC_ROUND_ROWS * DC_WARPS * 8;
+    red = (size_t)3 * DC_ROUND_ROWS * DC_WARPS * 8;
   }
   const size_t limit = 227 * 1024;
+  auto total = [&](int nt) { return act + ring + std::max((size_t)nt * p.tab_bytes, stage) + red; };
   p.ntabs = (int)std::max<size_t>(2, std::min<size_t>(DC_MAX_TABS, DC_TAB_BUDGET / p.tab_bytes));
-  while (p.ntabs > 2 && act + ring + std::max((size_t)p.ntabs * p.tab_bytes, over) > limit) --p.ntabs;
+  while (p.ntabs > 2 && total(p.ntabs) > limit) --p.ntabs;
   p.nfold = std::min(p.ntabs, DC_FOLD_WARPS);
   p.ntabs -= p.ntabs % p.nfold;
-  const size_t smem = act + ring + std::max((size_t)p.ntabs * p.tab_bytes, over);
+  p.red_off = (int)(p.tab_off + std::max((size_t)p.ntabs * p.tab_bytes, stage));
+  const size_t smem = total(p.ntabs);
   if (smem > limit) return cudaErrorInvalidValue;
 #define BWTA_DC(R)                                                                              \
   return fused ? launch_decode_t<R, true>(p, smem, d_status, s)                                 \
