@@ -180,8 +180,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-// Bounded wait that also records a timeout for the whole CTA.
+// Bounded wait that also records a timeout for the whole CTA. A phase that
+// has already completed (the usual case in the tile loops) is seen by one
+// non-blocking test, without entering the suspending wait.
 __device__ __forceinline__ bool dc_wait(DcBars &b, uint64_t *bar, uint32_t parity) {
+  if (mbar_test(bar, parity)) return true;
   if (*(volatile int32_t *)&b.timeout) return false;
   if (mbar_wait(bar, parity, 2000000000ull)) return true;
   b.timeout = 1;
