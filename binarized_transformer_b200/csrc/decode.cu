@@ -13,23 +13,25 @@
 // -- the same fp32 operations, in the same order, as the tiled GEMM, so the
 // outputs agree bit for bit.
 //
-// Work is cut into tiles of DC_R = 16 weight rows of one projection; a CTA
-// takes tiles blockIdx.x, blockIdx.x + gridDim.x, ... (all of a tile's K at
-// once). Warp roles:
+// Work is cut into tiles of R weight rows of one projection (R = 32 when two
+// such tiles fit the copy ring and at most two activation rows are batched,
+// else 16); a CTA takes tiles blockIdx.x, blockIdx.x + gridDim.x, ... (all
+// of a tile's K at once). Every wait and release below is per tile, so the
+// taller tile halves their count per row. Warp roles:
 //  * the copy warp (one thread) brings each tile into a ring of shared-memory
 //    stages with two bulk copies -- the tile's rows of sign words are one
 //    contiguous block (rows are ldw words apart), and so are its rows of
 //    weight scales -- completing on the stage's mbarrier; with the weights
 //    known to be complete it fills the ring before the kernel waits for the
 //    previous kernel in the stream;
-//  * eight dot warps compute the integer dots: warp w takes rows 2w and
-//    2w + 1 of the tile, lane c the 128-element chunks c, c + 32, ... (16
+//  * eight dot warps compute the integer dots: warp w takes rows R/8 w ...
+//    R/8 (w + 1) - 1 of the tile, lane c the 128-element chunks c, c + 32, ... (16
 //    contiguous bytes per lane, conflict-free), and write each chunk's dot
 //    (int16: |d| <= 128) and weight scale to a fold table [row][chunk] with an
 //    odd row pitch, then release the stage;
 //  * four fold warps take the tiles in turn (tile i: fold warp i mod 4):
 //    lane r walks row r's chunks in order (integer group sums, one fma per
-//    group) and writes Y -- reads at an odd pitch, so the 16 lanes hit 16
+//    group) and writes Y -- reads at an odd pitch, so the R lanes hit R
 //    banks. The fold is a serial chain per row; keeping it off the dot warps
 //    lets them run ahead by as many tiles as there are fold tables.
 // The activation planes of every job sit in shared memory for the whole
@@ -51,8 +53,6 @@ constexpr int DC_CTHREADS = DC_WARPS * 32;       // dot threads (named barrier 1
 constexpr int DC_FOLD_WARPS = 4;                 // fold warps
 constexpr int DC_COPY_WARP = DC_WARPS + DC_FOLD_WARPS;
 constexpr int DC_THREADS = (DC_COPY_WARP + 1) * 32;
-constexpr int DC_R = 16;                         // weight rows per tile
-constexpr int DC_RPW = DC_R / DC_WARPS;          // rows per dot warp
 constexpr int DC_MAX_STAGES = 16;
 constexpr int DC_MAX_TABS = 8;
 constexpr int DC_MAX_JOBS = 8;
@@ -65,7 +65,6 @@ constexpr size_t DC_RING_BUDGET = 56 * 1024;     // bytes of weight tiles in fli
 constexpr size_t DC_TAB_BUDGET = 48 * 1024;      // fold tables (at least two)
 constexpr int DC_STAGE_ROWS_BYTES = 48 * 1024;   // fused: fp16 rows staged per round
 constexpr int DC_ROUND_ROWS = 32;                // fused: at most this many rows per round
-static_assert(DC_R == 16 && DC_RPW * DC_WARPS == DC_R, "fold lanes 0..15, two rows per warp");
 
 struct DecodeJob {
   const uint16_t *X;            // fused: fp16 rows [M][ldX]
@@ -80,6 +79,7 @@ struct DecodeJob {
   int64_t ldY;
   int32_t *dots;
   int64_t ldD;
+  double inv2k;                 // fused: 1 / (2 K), the threshold's divisor as a reciprocal
   int64_t tile0;                // first global tile of this job
   int M, nchunks, gchunks;
   int act_off;                  // byte offset of the job's planes in shared memory
@@ -155,8 +155,8 @@ struct DcCursor {
       tend = j + 1 < p.njobs ? p.job[j + 1].tile0 : p.ntiles;
     }
   }
-  // rows of the tile that starts at row n0 (the job's last tile may be short)
-  __device__ __forceinline__ int64_t rows(int64_t n0) const { return N - n0 < DC_R ? N - n0 : DC_R; }
+  // rows of the tile of R rows that starts at row n0 (the job's last tile may be short)
+  __device__ __forceinline__ int64_t rows(int64_t n0, int R) const { return N - n0 < R ? N - n0 : R; }
 };
 
 // Bulk copy global -> this CTA's shared memory (no multicast), completing on
@@ -202,6 +202,20 @@ __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
   const uint64_t mid = __reduce_add_sync(FULL, (uint32_t)((v >> 22) & L22));
   const uint64_t hi = __reduce_add_sync(FULL, (uint32_t)(v >> 44));
   return lo + (mid << 22) + (hi << 44);
+}
+
+// floor(S / d) for d = 2K: S is a sum of K magnitudes below 2^40 units, so the
+// quotient is below 2^39 and the fp64 estimate S * (1/d) is within 2^-12 of
+// it; one integer correction step in either direction makes it exact (a 64-bit
+// integer division is a long dependent subroutine on the setup's critical
+// path).
+__device__ __forceinline__ uint64_t floor_div_2k(uint64_t S, int64_t d, double inv_d) {
+  if (d <= 0) return 0;  // an empty row: no element to threshold
+  uint64_t q = (uint64_t)__dmul_rz(__ull2double_rn(S), inv_d);
+  const uint64_t ud = (uint64_t)d;
+  if (q * ud > S) --q;
+  else if (S - q * ud >= ud) ++q;
+  return q;
 }
 
 // Planes of every job into shared memory: copied (bit-plane input) or made
@@ -307,7 +321,7 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
         uint64_t S = 0;
 #pragma unroll
         for (int w = 0; w < DC_WARPS; ++w) S += red_s[r * DC_WARPS + w];
-        const uint32_t hT = p.ternary ? mag_threshold_pattern(S / (uint64_t)(2 * K)) : 0u;
+        const uint32_t hT = p.ternary ? mag_threshold_pattern(floor_div_2k(S, 2 * K, J.inv2k)) : 0u;
         uint4 *sA = reinterpret_cast<uint4 *>(smem + J.act_off);
         uint32_t *mrow = reinterpret_cast<uint32_t *>(sA + mm * nch);
         uint32_t *srow = reinterpret_cast<uint32_t *>(sA + J.M * nch + mm * nch);
@@ -372,15 +386,15 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
 }
 
 // ------------------------------------------------------------------ kernel
-// Fold table b: d [MR][DC_R][pitch] int16, then alpha [DC_R][pitch] fp32.
-__host__ __device__ __forceinline__ size_t dc_tab_d_bytes(int mr, int pitch) {
-  return ((size_t)mr * DC_R * pitch * 2 + 15) / 16 * 16;
+// Fold table b: d [MR][R][pitch] int16, then alpha [R][pitch] fp32.
+__host__ __device__ __forceinline__ size_t dc_tab_d_bytes(int mr, int R, int pitch) {
+  return ((size_t)mr * R * pitch * 2 + 15) / 16 * 16;
 }
 
 // Two CTAs per SM by registers: an SM running a CTA of this launch keeps room
 // for a CTA of the next kernel in the stream (416 threads x 80 registers, the
 // allocation of 74, would not fit twice in 64 K registers).
-template <int MR, bool FUSED>
+template <int MR, bool FUSED, int R>
 __global__ void __launch_bounds__(DC_THREADS, 2)
 k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
   extern __shared__ uint4 dc_smem4[];
@@ -395,6 +409,8 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
     reinterpret_cast<uint32_t *>(&p_s)[w] = reinterpret_cast<const uint32_t *>(&pk)[w];
   __syncthreads();
   const DecodeBatch &p = p_s;
+  static_assert((R == 16 || R == 32) && R % DC_WARPS == 0, "fold lanes 0..R-1, R/8 rows per dot warp");
+  constexpr int RPW = R / DC_WARPS;  // rows per dot warp
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t stride = gridDim.x;
   uint8_t *ring = smem + p.ring_off;
@@ -434,8 +450,8 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
       for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += stride, ++i) {
         if (i >= p.stages && !dc_wait(bars, &bars.empty[s], (round & 1) ^ 1)) break;
         c.seek(p, tile);
-        const int64_t n0 = (tile - c.t0) * DC_R;
-        const int64_t rows = c.rows(n0);
+        const int64_t n0 = (tile - c.t0) * R;
+        const int64_t rows = c.rows(n0, R);
         uint8_t *st = ring + (size_t)s * p.stage_bytes;
         const uint32_t bbytes = (uint32_t)(rows * c.ldw * 4);
         const uint32_t sbytes = c.Y ? (uint32_t)(rows * c.G * 4) : 0u, s16 = sbytes & ~15u;
@@ -452,7 +468,7 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
         // once the ring's first fill is out, keep tiles i+1 .. i+pf_ahead prefetched
         for (; i + 1 >= p.stages && pi <= i + p.pf_ahead && ptile < p.ntiles; ptile += stride, ++pi) {
           pc.seek(p, ptile);
-          const int64_t m0 = (ptile - pc.t0) * DC_R, prow = pc.rows(m0);
+          const int64_t m0 = (ptile - pc.t0) * R, prow = pc.rows(m0, R);
           bulk_prefetch_l2(pc.wb + m0 * pc.ldw, (uint32_t)(prow * pc.ldw * 4), pol);
           const uint32_t ps16 = pc.Y ? (uint32_t)(prow * pc.G * 4) & ~15u : 0u;
           if (ps16) bulk_prefetch_l2(pc.ws + m0 * pc.G, ps16, pol);
@@ -491,12 +507,12 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
       const JobActs acts = job_acts(smem, J);
       const uint8_t *tab = smem + p.tab_off + (size_t)b * p.tab_bytes;
       const int nch = J.nchunks, gc = J.gchunks;
-      const int64_t n = (tile - J.tile0) * DC_R + lane;
-      if (lane < DC_R) {
+      const int64_t n = (tile - J.tile0) * R + lane;
+      if (lane < R) {
         // lane r walks row r's chunks in order
         const int16_t *dr = reinterpret_cast<const int16_t *>(tab) + lane * p.pitch;
-        const float *ar = reinterpret_cast<const float *>(tab + dc_tab_d_bytes(MR, p.pitch)) + lane * p.pitch;
-        const int dstride = DC_R * p.pitch;
+        const float *ar = reinterpret_cast<const float *>(tab + dc_tab_d_bytes(MR, R, p.pitch)) + lane * p.pitch;
+        const int dstride = R * p.pitch;
         float acc[MR];
         int dt[MR], gd[MR];
 #pragma unroll
@@ -596,41 +612,44 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
     const uint8_t *st = ring + (size_t)s * p.stage_bytes;
     uint8_t *tab = smem + p.tab_off + (size_t)b * p.tab_bytes;
     int16_t *td = reinterpret_cast<int16_t *>(tab);
-    float *ta = reinterpret_cast<float *>(tab + dc_tab_d_bytes(MR, p.pitch));
-    // integer dots of this warp's two rows with every activation row. The
+    float *ta = reinterpret_cast<float *>(tab + dc_tab_d_bytes(MR, R, p.pitch));
+    // integer dots of this warp's RPW rows with every activation row. The
     // rows share each activation chunk's loads, and all of a chunk's loads are
     // issued before its stores (a store to the table may alias a later load,
     // so the compiler keeps them in program order).
-    static_assert(DC_RPW == 2, "two rows per dot warp");
-    const int r0 = warp * DC_RPW;
-    const uint4 *bits0 = reinterpret_cast<const uint4 *>(st + (size_t)r0 * jldw * 4);
-    const uint4 *bits1 = reinterpret_cast<const uint4 *>(st + (size_t)(r0 + 1) * jldw * 4);
+    const int r0 = warp * RPW;
+    const uint8_t *bits0 = st + (size_t)r0 * jldw * 4;
     const float *sc0 = reinterpret_cast<const float *>(st + p.stage_bits) + r0 * jG;
-    const float *sc1 = sc0 + jG;
     for (int c = lane; c < nch; c += 32) {
-      const uint4 w0 = bits0[c], w1 = bits1[c];
       const int g = gc == 1 ? c : c / gc;
-      const float a0 = jY ? sc0[g] : 0.0f, a1 = jY ? sc1[g] : 0.0f;
-      int d0[MR], d1[MR];
+      uint4 w[RPW];
+      float a[RPW];
+#pragma unroll
+      for (int q = 0; q < RPW; ++q) {
+        w[q] = reinterpret_cast<const uint4 *>(bits0 + (size_t)q * jldw * 4)[c];
+        a[q] = jY ? sc0[q * jG + g] : 0.0f;
+      }
+      int d[RPW][MR];
 #pragma unroll
       for (int m = 0; m < MR; ++m) {
-        d0[m] = d1[m] = 0;
         if (m < jM) {
           const uint4 A = acts.sA[m * nch + c], S = acts.sS[m * nch + c];
           const int P = acts.sP[m * nch + c];
-          d0[m] = P - 2 * popc4_csa(lop3_and_xor(A.x, S.x, w0.x), lop3_and_xor(A.y, S.y, w0.y),
-                                    lop3_and_xor(A.z, S.z, w0.z), lop3_and_xor(A.w, S.w, w0.w));
-          d1[m] = P - 2 * popc4_csa(lop3_and_xor(A.x, S.x, w1.x), lop3_and_xor(A.y, S.y, w1.y),
-                                    lop3_and_xor(A.z, S.z, w1.z), lop3_and_xor(A.w, S.w, w1.w));
+#pragma unroll
+          for (int q = 0; q < RPW; ++q)
+            d[q][m] = P - 2 * popc4_csa(lop3_and_xor(A.x, S.x, w[q].x), lop3_and_xor(A.y, S.y, w[q].y),
+                                        lop3_and_xor(A.z, S.z, w[q].z), lop3_and_xor(A.w, S.w, w[q].w));
+        } else {
+#pragma unroll
+          for (int q = 0; q < RPW; ++q) d[q][m] = 0;
         }
       }
-      ta[r0 * p.pitch + c] = a0;
-      ta[(r0 + 1) * p.pitch + c] = a1;
 #pragma unroll
-      for (int m = 0; m < MR; ++m) {
-        td[(m * DC_R + r0) * p.pitch + c] = (int16_t)d0[m];
-        td[(m * DC_R + r0 + 1) * p.pitch + c] = (int16_t)d1[m];
-      }
+      for (int q = 0; q < RPW; ++q) ta[(r0 + q) * p.pitch + c] = a[q];
+#pragma unroll
+      for (int m = 0; m < MR; ++m)
+#pragma unroll
+        for (int q = 0; q < RPW; ++q) td[(m * R + r0 + q) * p.pitch + c] = (int16_t)d[q][m];
     }
     __syncwarp();
     if (lane == 0) {
@@ -661,10 +680,10 @@ bool decode_fits(int64_t M, int64_t K) {
          dc_act_bytes((int)M, (int)nchunks) <= DC_MAX_ACT_SMEM;
 }
 
-template <int MR, bool FUSED>
+template <int MR, bool FUSED, int R>
 static cudaError_t launch_decode_t(const DecodeBatch &p, size_t smem, int32_t *d_status,
                                    cudaStream_t s) {
-  auto kern = k_decode<MR, FUSED>;
+  auto kern = k_decode<MR, FUSED, R>;
   static SmemOptIn opt_in;
   if (cudaError_t e = opt_in(kern, (int)smem, true)) return e;
   int dev = 0, sms = 148;
@@ -703,6 +722,7 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
     J.ldY = in.ldY;
     J.dots = in.dots;
     J.ldD = in.ldD;
+    J.inv2k = 1.0 / (2.0 * (double)in.K);
     J.M = (int)in.M;
     J.nchunks = (int)ceil_div<int64_t>(ceil_div<int64_t>(in.K, 32), 4);
     J.gchunks = in.group ? (int)(in.group / 128) : J.nchunks;
@@ -710,8 +730,6 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
     J.vec = (reinterpret_cast<uintptr_t>(in.X) & 15u) == 0 && in.ldX % 8 == 0;
     J.act_off = (int)act;
     act += dc_act_bytes(J.M, J.nchunks);
-    J.tile0 = p.ntiles;
-    p.ntiles += ceil_div<int64_t>(in.N, DC_R);
     MR = std::max(MR, J.M);
     nch_max = std::max(nch_max, J.nchunks);
     ldw_max = std::max(ldw_max, J.ldw);
@@ -724,9 +742,17 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
   p.ternary = mode == BWTA_TERNARY;
   p.ready = ready;
   const int mr = MR <= 1 ? 1 : MR <= 2 ? 2 : MR <= 4 ? 4 : 8;
-  // copy ring: DC_R rows of sign words and of scales of the widest job
-  p.stage_bits = (int)(DC_R * ldw_max * 4);
-  p.stage_bytes = (int)((p.stage_bits + DC_R * G_max * 4 + 15) / 16 * 16);
+  // tile height: 32 rows where two such tiles of the widest job fit the copy
+  // ring and the dot warps' registers hold 4 rows x MR dots
+  auto stage_of = [&](int64_t R) { return (R * ldw_max * 4 + R * G_max * 4 + 15) / 16 * 16; };
+  const int R = (mr <= 2 && 2 * (size_t)stage_of(32) <= DC_RING_BUDGET) ? 32 : 16;
+  for (int i = 0; i < nj; ++i) {
+    p.job[i].tile0 = p.ntiles;
+    p.ntiles += ceil_div<int64_t>(p.job[i].N, R);
+  }
+  // copy ring: R rows of sign words and of scales of the widest job
+  p.stage_bits = (int)(R * ldw_max * 4);
+  p.stage_bytes = (int)stage_of(R);
   p.stages = (int)std::min<size_t>(DC_MAX_STAGES,
                                    std::max<size_t>(2, DC_RING_BUDGET / (size_t)p.stage_bytes));
   // L2 prefetch window: about DC_PF_BYTES of tiles per CTA beyond the ring
@@ -737,7 +763,7 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
   // after both (read by the scale threads after the last barrier of the
   // setup, while other warps may already be writing fold tables)
   p.pitch = nch_max | 1;
-  p.tab_bytes = (int)((dc_tab_d_bytes(mr, p.pitch) + (size_t)DC_R * p.pitch * 4 + 15) / 16 * 16);
+  p.tab_bytes = (int)((dc_tab_d_bytes(mr, R, p.pitch) + (size_t)R * p.pitch * 4 + 15) / 16 * 16);
   p.tab_off = (int)(act + ring);
   size_t stage = 0, red = 0;
   if (fused) {  // every staged row fits; as many rows per round as the staging area holds
@@ -761,13 +787,15 @@ cudaError_t launch_decode(const DecodeSpec *jobs, int njobs, bool fused, int mod
   p.red_off = (int)(p.tab_off + std::max((size_t)p.ntabs * p.tab_bytes, stage));
   const size_t smem = total(p.ntabs);
   if (smem > limit) return cudaErrorInvalidValue;
-#define BWTA_DC(R)                                                                              \
-  return fused ? launch_decode_t<R, true>(p, smem, d_status, s)                                 \
-               : launch_decode_t<R, false>(p, smem, d_status, s)
-  if (mr == 1) BWTA_DC(1);
-  if (mr == 2) BWTA_DC(2);
-  if (mr == 4) BWTA_DC(4);
-  BWTA_DC(8);
+#define BWTA_DC(MRV, RV)                                                                        \
+  return fused ? launch_decode_t<MRV, true, RV>(p, smem, d_status, s)                           \
+               : launch_decode_t<MRV, false, RV>(p, smem, d_status, s)
+  if (mr == 1 && R == 32) BWTA_DC(1, 32);
+  if (mr == 2 && R == 32) BWTA_DC(2, 32);
+  if (mr == 1) BWTA_DC(1, 16);
+  if (mr == 2) BWTA_DC(2, 16);
+  if (mr == 4) BWTA_DC(4, 16);
+  BWTA_DC(8, 16);
 #undef BWTA_DC
 }
 

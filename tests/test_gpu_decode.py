@@ -60,6 +60,32 @@ def test_batched_mixed_jobs_exact(ready):
         check_job(X, W, group, Y.cpu().numpy(), D.cpu().numpy())
 
 
+# at most two activation rows and K small enough for two 32-row tiles in the
+# copy ring: the launch takes 32-row tiles; jobs end inside a tile (N = 1000,
+# 77) and one job has per-row scales
+TALL = [(1, 4096, 4096, 128), (2, 1000, 4096, 128), (1, 77, 2048, 0), (1, 11008, 4096, 128),
+        (2, 33, 300, 128)]
+
+
+@pytest.mark.parametrize("ready", [False, True])
+def test_batched_tall_tiles_exact(ready):
+    jobs, data = [], []
+    for i, (M, N, K, group) in enumerate(TALL):
+        X = workloads.edge_acts(M, K, "student", tag=200 + i)
+        W = workloads.edge_weights(N, K, tag=200 + i)
+        wb, ws = bt.bwta_pack_weights(dev(W), group)
+        jobs.append((dev(X), wb, ws, group))
+        data.append((X, W, group))
+    torch.cuda.synchronize()
+    st = bt.new_status()
+    outs = bt.bwta_linear_decode_batched(jobs, status=st, want_dots=True,
+                                         flags=bt.GEMM_WEIGHTS_READY if ready else 0)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    for (X, W, group), (Y, D) in zip(data, outs):
+        check_job(X, W, group, Y.cpu().numpy(), D.cpu().numpy())
+
+
 def test_batched_equals_single_calls():
     jobs, singles = [], []
     for i, (K, N) in enumerate(workloads.LLAMA_SHAPES):
