@@ -105,6 +105,7 @@ struct DcBars {
   uint64_t tfull[DC_MAX_TABS];    // the fold table is written (8 arrivals)
   uint64_t tempty[DC_MAX_TABS];   // the fold table is folded (1 arrival)
   int32_t timeout;
+  int32_t last_j0, last_m0, last_nr;  // fused: the rows of the last setup round (first job, row; count)
 };
 
 // Shared-memory planes of one job: sA [M][nchunks] uint4 (mask), sS (sign),
@@ -204,6 +205,50 @@ __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
   return lo + (mid << 22) + (hi << 44);
 }
 
+// The row scales of one setup round's nr rows (round row r = job jj, row mm,
+// counted from (j0, m0)), from the round's per-warp partial sums; thread t of
+// the calling group computes row t.
+__device__ __forceinline__ void dc_row_scales(const DecodeBatch &p, uint8_t *smem, int j0, int m0,
+                                              int nr, int t) {
+  if (t >= nr) return;
+  const uint64_t *red_s = reinterpret_cast<const uint64_t *>(smem + p.red_off);
+  const uint64_t *red_k = red_s + DC_ROUND_ROWS * DC_WARPS;
+  const uint64_t *red_n = red_k + DC_ROUND_ROWS * DC_WARPS;
+  int jj = j0, mm = m0;
+  for (int r = 0; r < t; ++r)
+    if (++mm == p.job[jj].M) {
+      mm = 0;
+      ++jj;
+    }
+  const DecodeJob &J = p.job[jj];
+  float *ssc = reinterpret_cast<float *>(smem + J.act_off + (size_t)J.M * J.nchunks * 36);
+  uint64_t a = 0, b = 0;
+  if (p.ternary) {
+#pragma unroll
+    for (int w = 0; w < DC_WARPS; ++w) {
+      a += red_k[t * DC_WARPS + w];
+      b += red_n[t * DC_WARPS + w];
+    }
+  } else {
+#pragma unroll
+    for (int w = 0; w < DC_WARPS; ++w) a += red_s[t * DC_WARPS + w];
+    b = (uint64_t)J.K;
+  }
+  ssc[mm] = row_scale(a, b);
+}
+
+// Named barriers of the fused setup's hand-off to the fold warps: the dot
+// warps arrive on DC_BAR_SETUP (without waiting) once the last round's
+// partial sums are written; the fold warps wait on it, make that round's row
+// scales, and meet on DC_BAR_FOLD before their first output.
+constexpr int DC_BAR_SETUP = 2, DC_BAR_FOLD = 3;
+__device__ __forceinline__ void bar_arrive_n(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void bar_sync_n(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // floor(S / d) for d = 2K: S is a sum of K magnitudes below 2^40 units, so the
 // quotient is below 2^39 and the fp64 estimate S * (1/d) is within 2^-12 of
 // it; one integer correction step in either direction makes it exact (a 64-bit
@@ -231,7 +276,8 @@ __device__ __forceinline__ uint64_t floor_div_2k(uint64_t S, int64_t d, double i
 // halves) of a row belongs to thread q % 256; 16 consecutive threads cover
 // one 128-element chunk.
 template <bool FUSED>
-__device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *smem, int32_t *d_status) {
+__device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *smem, DcBars &bars,
+                                              int32_t *d_status) {
   const int tid = threadIdx.x, wid = tid / 32, lane = tid % 32;
   if (!FUSED) {
     for (int j = 0; j < p.njobs; ++j) {
@@ -351,36 +397,23 @@ __device__ __forceinline__ void dc_setup_acts(const DecodeBatch &p, uint8_t *sme
         }
       }
     }
-    cbar();
-    // row scales (one thread per staged row)
-    if (tid < nr) {
-      int jj = j0, mm = m0;
-      for (int r = 0; r < tid; ++r)
-        if (++mm == p.job[jj].M) {
-          mm = 0;
-          ++jj;
-        }
-      const DecodeJob &J = p.job[jj];
-      float *ssc = reinterpret_cast<float *>(smem + J.act_off + (size_t)J.M * J.nchunks * 36);
-      uint64_t a = 0, b = 0;
-      if (p.ternary) {
-#pragma unroll
-        for (int w = 0; w < DC_WARPS; ++w) {
-          a += red_k[tid * DC_WARPS + w];
-          b += red_n[tid * DC_WARPS + w];
-        }
-      } else {
-#pragma unroll
-        for (int w = 0; w < DC_WARPS; ++w) a += red_s[tid * DC_WARPS + w];
-        b = (uint64_t)J.K;
+    if (j < p.njobs) {
+      // more rounds follow: this round's row scales now (one thread per row),
+      // before the staging area and the partial sums are reused
+      cbar();
+      dc_row_scales(p, smem, j0, m0, nr, tid);
+      cbar();
+    } else {
+      // the last round: its row scales are made by the fold warps (the only
+      // readers of scales), off the dot warps' way to their first tile
+      if (tid == 0) {
+        bars.last_j0 = j0;
+        bars.last_m0 = m0;
+        bars.last_nr = nr;
       }
-      ssc[mm] = row_scale(a, b);
+      bar_arrive_n(DC_BAR_SETUP, DC_CTHREADS + DC_FOLD_WARPS * 32);
+      cbar();  // every plane of the round is written before any dot warp reads one
     }
-    // The staging area and the partial sums are reused by the next round.
-    // After the last round no barrier is needed: the planes were complete at
-    // the barrier above, and the scales are read only by the fold warps,
-    // after the writer's warp has released its first fold table.
-    if (j < p.njobs) cbar();
   }
   if (bad) flag_status(d_status, BWTA_STATUS_NONFINITE);
 }
@@ -488,6 +521,13 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
   if (warp >= DC_WARPS) {
     // ------------------------------------------------ fold warps
     pdl_wait();  // outputs follow the previous kernel in the stream
+    if (FUSED) {
+      // the last setup round's row scales (the earlier rounds' are made by
+      // the dot warps), visible to every fold warp before its first output
+      bar_sync_n(DC_BAR_SETUP, DC_CTHREADS + DC_FOLD_WARPS * 32);
+      if (warp == DC_WARPS) dc_row_scales(p, smem, bars.last_j0, bars.last_m0, bars.last_nr, lane);
+      bar_sync_n(DC_BAR_FOLD, DC_FOLD_WARPS * 32);
+    }
     // Fold warp f takes tiles f, f + nfold, ...; with ntabs a multiple of
     // nfold, table b = i % ntabs is only ever folded by warp b % nfold, so
     // each table's barriers are waited on in order by one warp (a parity
@@ -589,7 +629,7 @@ k_decode(const __grid_constant__ DecodeBatch pk, int32_t *d_status) {
 
   // ------------------------------------------------ dot warps
   pdl_wait();  // activations follow the previous kernel in the stream
-  dc_setup_acts<FUSED>(p, smem, d_status);
+  dc_setup_acts<FUSED>(p, smem, bars, d_status);
 
   // stage and table indices and their rounds in counters; the current job's
   // fields in registers, reloaded when the tiles move into the next job
