@@ -93,12 +93,12 @@ def measured_peaks():
 
 # DRAM traffic of the tensor-core GEMM per launch, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum of the three prefill launches
-# of `bench.py --steps 2 --warmup 1`, averaged): 11.07, 43.87 and 29.72 MB for
+# of `bench.py --steps 2 --warmup 1`, averaged): 11.07, 45.36 and 29.89 MB for
 # K x N = 4096x4096, 4096x11008, 11008x4096 at M = 2048. Valid only for the
 # kernel source it was taken on; reported as null once that file changes.
 TC_TRAFFIC = {"source": "binarized_transformer_b200/csrc/gemm_tc.cu",
-              "sha256": "8aefdc421c9c3d65532d7ae9fab9b47dad4ec67eb95233abdef1db62843cc791",
-              "bytes_per_launch": 28779435}
+              "sha256": "8e7c93859df902da794099f85b99b4b2f2fca0f374fb2a490df91bffd3fb50b7",
+              "bytes_per_launch": 28772693}
 
 
 def tc_traffic():

@@ -21,15 +21,20 @@
 //    lane per weight row, 4 buffers). Weight k + 8j of a 32-column block goes
 //    to byte j of word k, the order in which the activation packer writes its
 //    E4M3 bytes, so a word costs one shift and one LOP3;
-//  * warp 1 (one thread) issues 4 MMAs (M=128, N=128, K=32) per k-block into
-//    one of three fp32 accumulators in TMEM (one per weight group in flight);
+//  * warps 1 and 14 (one thread each) issue 4 MMAs (M=128, N=128, K=32) per
+//    k-block into one of three fp32 accumulators in TMEM (one per weight
+//    group in flight); with groups of one or two k-blocks issuer i takes the
+//    groups with index = i (mod 2), so every MMA of a group comes from one
+//    thread, in order; with longer groups warp 1 issues them all;
 //  * warps 6-13 fold each finished group into running fp32 sums in registers
 //    (two warps per TMEM lane quarter, 64 tokens each) and write Y at the end
 //    of a tile.
 // MMA issue blocks until the tensor pipe takes the instruction, and the pipe
 // takes the next MMA only as the previous one finishes (64 cycles for
-// M=128, N=128, K=32), so every gap in the issuing thread is idle pipe time.
-// It does as little as possible between MMAs: one commit per k-block, into a
+// M=128, N=128, K=32), so every gap in an issuing thread is idle pipe time.
+// Two issuers on different SM sub-partitions keep the pipe fed through each
+// other's gaps, and each does as little as possible between MMAs: one commit
+// per k-block, into a
 // ring of "k-block done" barriers that frees the smem stage, the A buffer and
 // (for groups of at most two k-blocks) signals the finished accumulator all
 // at once; the barriers of the next k-blocks are tested, without blocking,
@@ -53,15 +58,15 @@ constexpr int TC_STAGES = 8;    // smem ring of (activations, weight bits) k-blo
 constexpr int TC_ABUF = 4;      // expanded-weight buffers in TMEM
 constexpr int TC_DBUF = 3;      // fp32 accumulators in TMEM
 constexpr int TC_BATCH = 2;     // ready k-blocks issued back to back (<= TC_DBUF)
-// Warps: 0 TMA, 1 MMA issue, 2-5 expand, 6-13 epilogue. A warp reaches the
+// Warps: 0 TMA, 1 and 14 MMA issue, 2-5 expand, 6-13 epilogue. A warp reaches the
 // TMEM lanes of quarter warp % 4 only, so the expand and epilogue warps cover
 // the four quarters by their index mod 4. The MMA issuer shares its SM
 // sub-partition with busy expand and epilogue warps; measured alone, its MMA
 // rate drops 3.6x when high-ILP warps compete for the same issue slots, so it
 // is the lowest-numbered warp there and the epilogue issues half as many FMA
 // instructions (two fp32 FMAs per instruction).
-constexpr int TC_PRODUCER = 0, TC_ISSUER = 1, TC_EXPAND0 = 2, TC_EPI0 = 6;
-constexpr int TC_THREADS = 14 * 32;
+constexpr int TC_PRODUCER = 0, TC_ISSUER = 1, TC_EXPAND0 = 2, TC_EPI0 = 6, TC_ISSUER2 = 14;
+constexpr int TC_THREADS = 15 * 32;
 constexpr int TC_X_BYTES = TC_BN * TC_KB;  // 16 KB of E4M3 activations per stage
 constexpr int TC_W_BYTES = TC_BM * 16;     // 2 KB of weight sign bits per stage
 constexpr int TC_STAGE_BYTES = TC_X_BYTES + TC_W_BYTES;
@@ -76,7 +81,19 @@ static_assert(TC_STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned");
 // provides after its wait: the producer's load (always), the expand warps'
 // A buffer (TC_STAGES >= TC_ABUF) and the epilogue's accumulator release
 // (groups of seg_len k-blocks with TC_STAGES >= TC_DBUF * seg_len; longer
-// groups get their own commit on d_full).
+// groups get their own commit on d_full). A commit tracks the MMAs of its own
+// thread, and every wait names the k-block whose MMAs it needs.
+// Two issuers: an issuer waits on full[] and a_full[] for its k-blocks only,
+// skipping the other's. A parity wait for k-block g is sound when the slot's
+// previous phase (k-block g - TC_STAGES, resp. g - TC_ABUF) has completed, and
+// that holds when that k-block is the same issuer's (it waited for it). With
+// groups of seg_len k-blocks handed out alternately, g - R is the same
+// issuer's for every g exactly when R / seg_len is even: seg_len 1 or 2 for
+// R = 4 and 8. Longer groups (up to a whole K) would let an issuer find a
+// phase of the same parity from two rounds before, so they run on one issuer.
+constexpr int TC_DUAL_MAX_GROUP = 2;
+static_assert(TC_ABUF % (2 * TC_DUAL_MAX_GROUP) == 0 && TC_STAGES % (2 * TC_DUAL_MAX_GROUP) == 0,
+              "two issuers need whole pairs of groups in every ring");
 static_assert(TC_STAGES >= TC_ABUF && TC_STAGES >= 2 * TC_DBUF, "ring sizes");
 constexpr int TC_SHORT_GROUP = TC_STAGES / TC_DBUF;  // longest group signalled through done[]
 
@@ -175,7 +192,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
       mbar_init(&bars->d_full[i], 1);
       mbar_init(&bars->d_empty[i], 8);
     }
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain, 2);  // one commit per issuer
     bars->timeout = 0;
     bars->undrained = 0;
     mbar_fence_init();
@@ -219,9 +236,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
           bars->undrained = 1;
     }
     __syncwarp();
-  } else if (warp == TC_ISSUER) {
+  } else if (warp == TC_ISSUER || warp == TC_ISSUER2) {
     // ------------------------------------------------ MMA issue
     if (lane == 0) {
+      const uint32_t me = warp == TC_ISSUER ? 0u : 1u;  // this issuer's groups: sg % 2 == me
+      const bool dual = seg_len <= TC_DUAL_MAX_GROUP;    // else warp 1 issues every group
       const uint32_t idesc = idesc_e4m3_f32(TC_BM, TC_BN);
       // Non-blocking test of everything k-block c needs.
       auto ready = [&](const TcCursor &c) -> bool {
@@ -250,8 +269,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
         tc_commit(&bars->done[c.g % TC_STAGES]);
         if (c.last && !short_group) tc_commit(&bars->d_full[d]);
       };
+      // Step c to this issuer's next k-block (or past the last tile).
+      auto own = [&](TcCursor &c) {
+        while (dual && c.tile < ntiles && (c.sg & 1u) != me) c.advance(KB, seg_len, gridDim.x);
+      };
       TcCursor cur{(int64_t)blockIdx.x, 0, 0, 0u, 0u, true, true};
       cur.set_flags(KB, seg_len);
+      if (!dual && me == 1) cur.tile = ntiles;  // nothing to issue
+      own(cur);
       bool rdy = cur.tile < ntiles && ready(cur);
       while (cur.tile < ntiles) {
         if (!rdy && !wait_all(cur)) break;
@@ -265,9 +290,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
         int nb = 1;
         TcCursor nxt = cur;
         nxt.advance(KB, seg_len, gridDim.x);
+        own(nxt);
         while (nb < TC_BATCH && nxt.tile < ntiles && ready(nxt)) {
           batch[nb++] = nxt;
           nxt.advance(KB, seg_len, gridDim.x);
+          own(nxt);
         }
         tc_fence_after();
 #pragma unroll
@@ -276,12 +303,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUt
         cur = nxt;
         rdy = cur.tile < ntiles && ready(cur);
       }
-      // Every MMA issued has completed before TMEM is released.
+      // Every MMA issued (by both issuers) has completed before TMEM is released.
       tc_commit(&bars->drain);
       if (!mbar_wait(&bars->drain, 0, DRAIN_NS)) bars->undrained = 1;
     }
     __syncwarp();
-  } else if (warp < TC_EPI0) {
+  } else if (warp >= TC_EXPAND0 && warp < TC_EPI0) {
     // ------------------------------------------------ weight bits -> E4M3 in TMEM
     const int qx = warp % 4, r = qx * 32 + lane;
     uint32_t g = 0;
