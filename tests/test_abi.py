@@ -97,6 +97,89 @@ def test_validation_rejects_before_launch(lib):
     assert lib.billm_gemm(FAKE, 1, 256, None, FAKE, 4, None, None) == E.BWTA_ERR_INVALID_ARG
 
 
+def test_validation_of_the_fused_and_tensor_core_calls(lib):
+    """The packer with E4M3 output, the tensor-core GEMM, the fused decode
+    (single and batched) and the attention calls past the scores reject bad
+    arguments, and accept empty problems, without any launch."""
+    import binarized_transformer_b200 as bt
+    E = bt
+    nan = float("nan")
+    # bwta_quantize_pack_acts_ex: half a plane pair, no output, short or
+    # misaligned E4M3 rows, ratio, plane stride
+    qx = lib.bwta_quantize_pack_acts_ex
+    assert qx(FAKE, 2, 256, 256, 0, 0.5, FAKE, None, 8, None, 0, FAKE, None, None) == E.BWTA_ERR_INVALID_ARG
+    assert qx(FAKE, 2, 256, 256, 0, 0.5, None, None, 8, None, 0, FAKE, None, None) == E.BWTA_ERR_INVALID_ARG
+    assert qx(FAKE, 2, 256, 256, 0, 0.5, None, None, 8, FAKE, 128, FAKE, None, None) == E.BWTA_ERR_INVALID_ARG
+    assert qx(FAKE, 2, 256, 256, 0, 0.5, None, None, 8, MISALIGNED, 256, FAKE, None, None) == \
+        E.BWTA_ERR_ALIGNMENT
+    assert qx(FAKE, 2, 256, 256, 0, 0.5, None, None, 8, FAKE, 264, FAKE, None, None) == E.BWTA_ERR_ALIGNMENT
+    assert qx(FAKE, 2, 256, 256, 0, 0.3, None, None, 8, FAKE, 256, FAKE, None, None) == E.BWTA_ERR_UNSUPPORTED
+    assert qx(FAKE, 2, 256, 256, 0, 0.5, FAKE, FAKE, 10, None, 0, FAKE, None, None) == E.BWTA_ERR_ALIGNMENT
+    # bwta_gemm_tc: no outputs, group, K bound, E4M3 row stride and alignment,
+    # weight-plane stride; an empty problem returns OK without a launch
+    tc = lib.bwta_gemm_tc
+    assert tc(FAKE, 256, FAKE, 4, FAKE, FAKE, 4, 8, 256, 0, None, 4, None, 4, None, None) == \
+        E.BWTA_ERR_INVALID_ARG
+    assert tc(FAKE, 256, FAKE, 4, FAKE, FAKE, 4, 8, 256, 100, FAKE, 4, None, 4, None, None) == \
+        E.BWTA_ERR_UNSUPPORTED
+    assert tc(FAKE, 256, FAKE, 4, FAKE, FAKE, 4, 8, (1 << 22) + 1, 0, FAKE, 4, None, 4, None, None) == \
+        E.BWTA_ERR_UNSUPPORTED
+    assert tc(FAKE, 128, FAKE, 4, FAKE, FAKE, 4, 8, 256, 0, FAKE, 4, None, 4, None, None) == \
+        E.BWTA_ERR_INVALID_ARG
+    assert tc(MISALIGNED, 256, FAKE, 4, FAKE, FAKE, 4, 8, 256, 0, FAKE, 4, None, 4, None, None) == \
+        E.BWTA_ERR_ALIGNMENT
+    assert tc(FAKE, 256, FAKE, 4, FAKE, FAKE, 4, 9, 256, 0, FAKE, 4, None, 4, None, None) == \
+        E.BWTA_ERR_ALIGNMENT
+    assert tc(None, 256, None, 0, FAKE, FAKE, 4, 8, 256, 0, FAKE, 4, None, 4, None, None) == E.BWTA_OK
+    # bwta_linear_decode: M > 8, K beyond the decode kernel, ldX < K, flags,
+    # ratio, mode, no outputs, misaligned weights
+    dc = lib.bwta_linear_decode
+    args = dict(X=FAKE, M=1, K=256, ldX=256, mode=0, r=0.5, wb=FAKE, ws=FAKE, N=4, ldw=8, g=128,
+                Y=FAKE, ldY=4, D=None, ldD=4, fl=0)
+
+    def dec(**kw):
+        a = dict(args, **kw)
+        return dc(a["X"], a["M"], a["K"], a["ldX"], a["mode"], a["r"], a["wb"], a["ws"], a["N"],
+                  a["ldw"], a["g"], a["Y"], a["ldY"], a["D"], a["ldD"], a["fl"], None, None)
+    assert dec(M=9) == E.BWTA_ERR_UNSUPPORTED
+    assert dec(K=16385, ldX=16385, ldw=516, g=0) == E.BWTA_ERR_UNSUPPORTED
+    assert dec(ldX=128) == E.BWTA_ERR_INVALID_ARG
+    assert dec(fl=2) == E.BWTA_ERR_INVALID_ARG
+    assert dec(r=0.25) == E.BWTA_ERR_UNSUPPORTED
+    assert dec(mode=7) == E.BWTA_ERR_INVALID_ARG
+    assert dec(Y=None) == E.BWTA_ERR_INVALID_ARG
+    assert dec(wb=MISALIGNED) == E.BWTA_ERR_ALIGNMENT
+    # bwta_linear_decode_batched: too many jobs, no descriptor array, the
+    # jobs' activation planes beyond the kernel's shared memory; all-empty
+    # jobs return OK without a launch
+    db = lib.bwta_linear_decode_batched
+
+    def jobs(*specs):
+        arr = (bt.DecodeJobC * len(specs))()
+        for i, (M, K, N) in enumerate(specs):
+            arr[i] = bt.DecodeJobC(0x10000, M, K, K, 0x10000, 0x10000, N, (K + 127) // 128 * 4, 128,
+                                   0x10000, N, None, N)
+        return arr
+    assert db(jobs(*[(1, 256, 4)] * 9), 9, 0, 0.5, 0, None, None) == E.BWTA_ERR_UNSUPPORTED
+    assert db(None, 1, 0, 0.5, 0, None, None) == E.BWTA_ERR_INVALID_ARG
+    assert db(jobs((8, 16384, 4), (8, 16384, 4)), 2, 0, 0.5, 0, None, None) == E.BWTA_ERR_UNSUPPORTED
+    assert db(jobs((0, 256, 4), (1, 256, 0)), 2, 0, 0.5, 0, None, None) == E.BWTA_OK
+    # bwta_attn_softmax_ternarize: no keys, wide rows, NaN scale, misaligned
+    # probability plane, missing probability scales
+    sm = lib.bwta_attn_softmax_ternarize
+
+    def soft(Lk=64, ld=4, scale=0.125, pm=FAKE, ps=FAKE):
+        return sm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, Lk, 64, ld, scale, pm, FAKE, 4, ps, None)
+    assert soft(Lk=0) == E.BWTA_ERR_INVALID_ARG
+    assert soft(ld=36) == E.BWTA_ERR_UNSUPPORTED
+    assert soft(scale=nan) == E.BWTA_ERR_UNSUPPORTED
+    assert soft(pm=MISALIGNED) == E.BWTA_ERR_ALIGNMENT
+    assert soft(ps=None) == E.BWTA_ERR_INVALID_ARG
+    # bwta_attn_av: no output
+    assert lib.bwta_attn_av(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 64, 64, 4, None, None, None) == \
+        E.BWTA_ERR_INVALID_ARG
+
+
 def test_binding_has_no_cpu_fallback():
     import torch
     import binarized_transformer_b200 as bt
